@@ -1,0 +1,131 @@
+/*
+ * squad.h - C ABI of libsquad, SQuad-Attention on NVIDIA B200 (sm_100a).
+ *
+ * The operator is the two-pass attention of "SQuad: Sub-Quadratic Attention
+ * Distillation for Efficient Video Generation" (gist.science technical
+ * summary, Methodology section 1, "SQuad-Attention Operator"; complexity claim
+ * O(n sqrt n) in the abstract):
+ *
+ *   tokens of a T x H x W latent grid, flattened p = (t*H + y)*W + x;
+ *   local pass  (per window of tT x tH x tW tokens, w = tT*tH*tW):
+ *       O1 = softmax(s * Q_w K_w^T) V_w
+ *   global pass (per group of the m = n/w tokens that share the same
+ *       in-window position (t mod tT, y mod tH, x mod tW)):
+ *       O  = softmax(s * Q_g K_g^T) O1_g
+ *   with the same input Q and K in both passes and s = 1/sqrt(d) unless the
+ *   caller gives another scale. The result is O (no residual, no mask).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, row-major [B, heads, n, d] with n = T*H*W (token
+ *     order as above); LSE vectors are [B, heads, n] float32, natural log.
+ *   - dtype SQUAD_BF16: q, k, v, o, o1, dout, dq, dk, dv are bfloat16 and the
+ *     kernels accumulate in fp32 (tcgen05 tensor cores). SQUAD_F32: all of
+ *     them are float32 and the kernels run fp32 FMA on the CUDA cores.
+ *   - Every pointer is a DEVICE pointer on the current CUDA device and must
+ *     be 16-byte aligned. The caller owns all memory; the library never
+ *     allocates, frees or synchronises in these calls. All work is enqueued
+ *     on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *   - Arguments are checked before anything is launched; on any error
+ *     nothing is enqueued. No entry point throws across the ABI.
+ */
+#ifndef SQUAD_H_
+#define SQUAD_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQUAD_OK = 0,
+  SQUAD_ERR_INVALID_ARG = 1,  /* NULL descriptor or required pointer, unknown dtype */
+  SQUAD_ERR_SHAPE = 2,        /* non-positive size, tile does not divide grid, size overflow */
+  SQUAD_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned */
+  SQUAD_ERR_UNSUPPORTED = 4,  /* valid operator, but outside what the kernels handle (see below) */
+  SQUAD_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed (see squad_last_cuda_error) */
+  SQUAD_ERR_TIMEOUT = 6,      /* a kernel gave up on a bounded wait (see squad_poll_device_error) */
+  SQUAD_ERR_WORKSPACE = 7     /* workspace missing or smaller than squad_attn_workspace_size */
+} squad_status;
+
+typedef enum { SQUAD_F32 = 0, SQUAD_BF16 = 1 } squad_dtype;
+
+typedef struct {
+  int B, heads, d;  /* batch, heads, head dimension */
+  int T, H, W;      /* latent grid; n = T*H*W */
+  int tT, tH, tW;   /* window tile; must divide T, H, W */
+  int dtype;        /* squad_dtype */
+  float scale;      /* softmax scale; <= 0 selects 1/sqrt(d) */
+} squad_desc;
+
+/* Limits of the kernels (SQUAD_ERR_UNSUPPORTED beyond them):
+ *   bf16: d in {64, 128}; tW <= 128 and W/tW <= 128 (a window row or a
+ *         group row must fit one 128-token tile); B*heads*n < 2^31.
+ *   f32:  d a multiple of 32, d <= 256; B*heads*n < 2^31.
+ * Any w and m are accepted otherwise (the bf16 kernels tile a window or a
+ * group into boxes of at most 128 tokens and run an online softmax across
+ * them). */
+
+/* Bytes of device workspace the call needs.
+ *   which = 0: squad_attn_fwd with o1 == NULL (the local-pass output is kept
+ *              there); with o1 != NULL the forward needs none.
+ *   which = 1: squad_attn_bwd (dO1 in the input dtype, the global-pass parts
+ *              of dQ and dK in fp32, and two fp32 row vectors).
+ * Returns SQUAD_OK and writes *bytes, or an argument/shape error. */
+squad_status squad_attn_workspace_size(const squad_desc* desc, int which, size_t* bytes);
+
+/* Forward: o = SQuad-Attention(q, k, v).
+ *   o1   : [B,heads,n,d] local-pass output, written when non-NULL (needed by
+ *          the backward); when NULL the workspace holds it.
+ *   lse1 : [B,heads,n] local-pass log-sum-exp, written when non-NULL.
+ *   lse2 : [B,heads,n] global-pass log-sum-exp, written when non-NULL.
+ *   workspace / workspace_bytes: see squad_attn_workspace_size(desc, 0, ..).
+ * Inputs must not alias outputs. */
+squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k, const void* v, void* o,
+                            void* o1, float* lse1, float* lse2, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* One pass of the forward, for callers that compose or time the passes on
+ * their own. stage 1 (local pass): out = per-window attention with values
+ * `val` = v. stage 2 (global pass): out = per-group attention with values
+ * `val` = the stage-1 output. lse (may be NULL) receives that pass's
+ * log-sum-exp. squad_attn_fwd is stage 1 followed by stage 2 on one stream. */
+squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* q, const void* k,
+                                 const void* val, void* out, float* lse, void* stream);
+
+/* Backward of the forward for the loss sum(o * dout): writes dq, dk, dv.
+ * o, o1, lse1, lse2 are the forward's outputs for the same q, k, v (all
+ * required). The global pass is differentiated first (values o1), then the
+ * local pass (values v); dq and dk sum both passes' contributions. */
+squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k, const void* v,
+                            const void* o, const void* o1, const float* lse1, const float* lse2,
+                            const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* Geometry the kernels use for one pass (stage 1 = local/window pass,
+ * stage 2 = global/cross-window pass), for tests and byte accounting.
+ * Writes 8 ints to info: [0] rows per problem (w or m), [1] problems per
+ * (batch, head), [2] tensor-core tiles per problem, [3] rows per tile box,
+ * [4] box extent along a, [5] along b, [6] along c, [7] key tiles held per
+ * online-softmax group. No CUDA call is made. */
+squad_status squad_plan_info(const squad_desc* desc, int stage, int* info);
+
+/* Synchronises `stream`, then reads and clears the library's device error
+ * word. Returns SQUAD_ERR_TIMEOUT if a kernel gave up on a bounded wait since
+ * the last poll, SQUAD_ERR_CUDA if the synchronisation failed, else SQUAD_OK. */
+squad_status squad_poll_device_error(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* squad_strerror(int status);
+
+/* cudaError_t / CUresult value of the last failing CUDA call on this thread. */
+int squad_last_cuda_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int squad_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQUAD_H_ */

@@ -1,0 +1,229 @@
+"""SQuad-Attention on NVIDIA B200: Python binding of the C-ABI library libsquad.
+
+The operator is the two-pass O(n sqrt n) attention of "SQuad: Sub-Quadratic
+Attention Distillation for Efficient Video Generation" (gist.science technical
+summary, Methodology section 1): softmax attention inside each tT x tH x tW
+window of a T x H x W token grid, then softmax attention across windows among
+tokens with the same in-window position, with the first pass's output as
+values. All arithmetic runs in the CUDA kernels of libsquad.so; this module
+only checks and marshals arguments (PyTorch supplies device memory and
+streams). There is no CPU fallback: without the built library every call
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "SquadError", "attention", "squad_attn_fwd", "squad_attn_bwd", "workspace_size",
+    "poll_device_error", "library_path", "load_library", "SQUAD_F32", "SQUAD_BF16", "squad_attn_fwd_pass",
+    "plan_info", "make_desc",
+]
+
+SQUAD_F32 = 0
+SQUAD_BF16 = 1
+_STATUS = {0: "SQUAD_OK", 1: "SQUAD_ERR_INVALID_ARG", 2: "SQUAD_ERR_SHAPE", 3: "SQUAD_ERR_ALIGN",
+           4: "SQUAD_ERR_UNSUPPORTED", 5: "SQUAD_ERR_CUDA", 6: "SQUAD_ERR_TIMEOUT", 7: "SQUAD_ERR_WORKSPACE"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class SquadError(RuntimeError):
+    def __init__(self, status: int, where: str, cuda_error: int = 0):
+        self.status = status
+        msg = f"{where}: {_STATUS.get(status, status)}"
+        if status == 5:
+            msg += f" (CUDA error {cuda_error})"
+        super().__init__(msg)
+
+
+class SquadDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("d", ctypes.c_int),
+                ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+                ("tT", ctypes.c_int), ("tH", ctypes.c_int), ("tW", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libsquad.so")
+
+
+def load_library():
+    """Load libsquad.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m sub_quadratic_two_b200.build`")
+        lib = ctypes.CDLL(path)
+        vp, sz, fp = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p
+        dp = ctypes.POINTER(SquadDesc)
+        lib.squad_attn_workspace_size.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+        lib.squad_attn_fwd.argtypes = [dp, vp, vp, vp, vp, vp, fp, fp, vp, sz, vp]
+        lib.squad_attn_bwd.argtypes = [dp, vp, vp, vp, vp, vp, fp, fp, vp, vp, vp, vp, vp, sz, vp]
+        lib.squad_attn_fwd_pass.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, fp, vp]
+        lib.squad_plan_info.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        lib.squad_poll_device_error.argtypes = [vp]
+        lib.squad_strerror.argtypes = [ctypes.c_int]
+        lib.squad_strerror.restype = ctypes.c_char_p
+        for f in ("squad_attn_workspace_size", "squad_attn_fwd", "squad_attn_bwd", "squad_poll_device_error",
+                  "squad_attn_fwd_pass", "squad_plan_info",
+                  "squad_last_cuda_error", "squad_version"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SquadError(status, where, load_library().squad_last_cuda_error())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SQUAD_F32
+    if t.dtype == torch.bfloat16:
+        return SQUAD_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def make_desc(q: torch.Tensor, grid: Sequence[int], tile: Sequence[int], scale: Optional[float]) -> SquadDesc:
+    if q.dim() != 4:
+        raise ValueError("expected [B, heads, n, d] tensors")
+    B, h, n, d = q.shape
+    T, H, W = (int(x) for x in grid)
+    tT, tH, tW = (int(x) for x in tile)
+    if T * H * W != n:
+        raise ValueError(f"n={n} but T*H*W={T * H * W}")
+    return SquadDesc(B, h, d, T, H, W, tT, tH, tW, _dtype_code(q), float(scale or 0.0))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], dev: torch.device):
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_inputs(*ts: torch.Tensor):
+    ref = ts[0]
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("libsquad needs CUDA tensors (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("libsquad needs contiguous [B, heads, n, d] tensors")
+        if t.dtype != ref.dtype or t.device != ref.device or t.shape != ref.shape:
+            raise ValueError("q, k, v (and gradients) must share shape, dtype and device")
+
+
+def workspace_size(desc: SquadDesc, which: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(load_library().squad_attn_workspace_size(ctypes.byref(desc), which, ctypes.byref(out)),
+           "squad_attn_workspace_size")
+    return int(out.value)
+
+
+def squad_attn_fwd(q, k, v, grid, tile, scale: Optional[float] = None, save: bool = True,
+                   stream: Optional[torch.cuda.Stream] = None, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None):
+    """Forward through the C ABI. Returns (o, o1, lse1, lse2); o1/lse are None when save=False.
+
+    With save=False the local-pass output lives in a workspace (``workspace``
+    if given, else a fresh allocation of ``workspace_size(desc, 0)`` bytes).
+    """
+    lib = load_library()
+    _check_inputs(q, k, v)
+    desc = make_desc(q, grid, tile, scale)
+    o = torch.empty_like(q) if out is None else out
+    if save:
+        o1 = torch.empty_like(q)
+        lse1 = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+        lse2 = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
+        ws, ws_bytes = None, 0
+    else:
+        o1 = lse1 = lse2 = None
+        ws_bytes = workspace_size(desc, 0)
+        ws = workspace if workspace is not None else torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        if ws.numel() * ws.element_size() < ws_bytes:
+            raise ValueError("workspace too small")
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.squad_attn_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o1), _ptr(lse1),
+                                  _ptr(lse2), _ptr(ws), ws_bytes, st), "squad_attn_fwd")
+    return o, o1, lse1, lse2
+
+
+def squad_attn_fwd_pass(stage: int, q, k, val, out, grid, tile, scale: Optional[float] = None,
+                        lse: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """One pass of the forward (stage 1: local, values V; stage 2: global, values O1) into ``out``."""
+    lib = load_library()
+    _check_inputs(q, k, val, out)
+    desc = make_desc(q, grid, tile, scale)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.squad_attn_fwd_pass(ctypes.byref(desc), int(stage), _ptr(q), _ptr(k), _ptr(val), _ptr(out),
+                                       _ptr(lse), st), "squad_attn_fwd_pass")
+    return out
+
+
+def plan_info(desc: SquadDesc, stage: int):
+    """Tiling of one pass: dict with rows, problems, tiles, box_rows, box (a, b, c), key_tiles_per_group."""
+    info = (ctypes.c_int * 8)()
+    _check(load_library().squad_plan_info(ctypes.byref(desc), int(stage), info), "squad_plan_info")
+    v = list(info)
+    return dict(rows=v[0], problems=v[1], tiles=v[2], box_rows=v[3], box=(v[4], v[5], v[6]), key_tiles_per_group=v[7])
+
+
+def squad_attn_bwd(q, k, v, o, o1, lse1, lse2, dout, grid, tile, scale: Optional[float] = None,
+                   stream: Optional[torch.cuda.Stream] = None):
+    """Backward through the C ABI. Returns (dq, dk, dv)."""
+    lib = load_library()
+    _check_inputs(q, k, v, o, o1, dout)
+    desc = make_desc(q, grid, tile, scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = workspace_size(desc, 1)
+    ws = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.squad_attn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o1),
+                                  _ptr(lse1.contiguous()), _ptr(lse2.contiguous()), _ptr(dout), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(ws), ws_bytes, st), "squad_attn_bwd")
+    return dq, dk, dv
+
+
+def poll_device_error(stream: Optional[torch.cuda.Stream] = None, device=None):
+    """Synchronise and raise SquadError(SQUAD_ERR_TIMEOUT) if a kernel gave up on a wait."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(load_library().squad_poll_device_error(_stream_handle(stream, dev)), "squad_poll_device_error")
+
+
+class _SquadAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, grid, tile, scale):
+        need = any(ctx.needs_input_grad[:3])
+        o, o1, lse1, lse2 = squad_attn_fwd(q, k, v, grid, tile, scale, save=need)
+        if need:
+            ctx.save_for_backward(q, k, v, o, o1, lse1, lse2)
+        ctx.geom = (tuple(grid), tuple(tile), scale)
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, o1, lse1, lse2 = ctx.saved_tensors
+        grid, tile, scale = ctx.geom
+        dq, dk, dv = squad_attn_bwd(q, k, v, o, o1, lse1, lse2, dout.contiguous(), grid, tile, scale)
+        return dq, dk, dv, None, None, None
+
+
+def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tuple[int, int, int],
+              tile: Tuple[int, int, int], scale: Optional[float] = None) -> torch.Tensor:
+    """SQuad-Attention of [B, heads, T*H*W, d] CUDA tensors (float32 or bfloat16), differentiable."""
+    return _SquadAttention.apply(q, k, v, tuple(grid), tuple(tile), scale)

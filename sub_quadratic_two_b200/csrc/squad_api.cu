@@ -1,0 +1,420 @@
+// squad_api.cu - the C ABI of libsquad (declared in include/squad.h).
+//
+// Host side only: argument checks, the per-pass geometry, TMA tensor maps and
+// kernel launches on the caller's stream. No allocation, no synchronisation
+// (except squad_poll_device_error, which says so).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "squad.h"
+#include "geometry.h"
+#include "squad_fwd_tc.cuh"
+#include "squad_simt.cuh"
+
+namespace {
+
+using sq::Geom;
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
+
+thread_local int t_last_cuda = 0;
+
+__device__ int g_squad_dev_err;  // set by kernels that gave up on a bounded wait
+
+squad_status cuda_fail(int code) {
+  t_last_cuda = code;
+  return SQUAD_ERR_CUDA;
+}
+
+#define SQ_CUDA(call)                                   \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(int(e_));   \
+  } while (0)
+
+// ---------------------------------------------------------------- per-device state
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;          // device address of g_squad_dev_err
+  bool fwd_attr_set[2][3] = {};  // [D=64/128][KT]
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+squad_status device_state(DeviceState** out) {
+  int dev = 0;
+  SQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return SQUAD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    SQ_CUDA(cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev));
+    void* p = nullptr;
+    SQ_CUDA(cudaGetSymbolAddress(&p, g_squad_dev_err));
+    s.err = static_cast<int*>(p);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+      SQ_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cuda_fail(int(cudaErrorSymbolNotFound));
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    s.ready = true;
+  }
+  *out = &s;
+  return SQUAD_OK;
+}
+
+// ---------------------------------------------------------------- argument checks
+
+struct Plan {
+  Geom g1, g2;        // local pass, global pass
+  long long rows;     // B*heads*n
+  size_t elem;        // bytes per element of q/k/v/o
+  float scale;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+squad_status make_plan(const squad_desc* d, Plan* p) {
+  if (d == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (d->dtype != SQUAD_F32 && d->dtype != SQUAD_BF16) return SQUAD_ERR_INVALID_ARG;
+  if (d->B <= 0 || d->heads <= 0 || d->d <= 0 || d->T <= 0 || d->H <= 0 || d->W <= 0 || d->tT <= 0 ||
+      d->tH <= 0 || d->tW <= 0)
+    return SQUAD_ERR_SHAPE;
+  if (d->T % d->tT || d->H % d->tH || d->W % d->tW) return SQUAD_ERR_SHAPE;
+  const long long n = (long long)d->T * d->H * d->W;
+  const long long rows = n * d->B * d->heads;
+  if (rows >= (1ll << 31) || rows * d->d >= (1ll << 40)) return SQUAD_ERR_SHAPE;
+  if (!(d->scale > 0.f) && !(d->scale <= 0.f)) return SQUAD_ERR_INVALID_ARG;  // NaN
+  if (d->dtype == SQUAD_BF16) {
+    if (d->d != 64 && d->d != 128) return SQUAD_ERR_UNSUPPORTED;
+  } else {
+    if (d->d % 32 != 0 || d->d > 256) return SQUAD_ERR_UNSUPPORTED;
+  }
+  p->g1 = sq::make_geom(1, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
+  p->g2 = sq::make_geom(2, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
+  if (d->dtype == SQUAD_BF16) {
+    if (!sq::plan_tiles(p->g1) || !sq::plan_tiles(p->g2)) return SQUAD_ERR_UNSUPPORTED;
+  }
+  p->rows = rows;
+  p->elem = d->dtype == SQUAD_BF16 ? 2 : 4;
+  p->scale = d->scale > 0.f ? d->scale : 1.0f / std::sqrt(float(d->d));
+  return SQUAD_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t fwd_workspace(const Plan& p, const squad_desc* d) { return align256(p.rows * d->d * p.elem); }
+
+struct BwdWs {
+  size_t do1, dq2, dk2, D2, D1, total;
+};
+
+BwdWs bwd_workspace(const Plan& p, const squad_desc* d) {
+  BwdWs w{};
+  const size_t big = p.rows * d->d;
+  w.do1 = 0;
+  w.dq2 = w.do1 + align256(big * p.elem);
+  w.dk2 = w.dq2 + align256(big * 4);
+  w.D2 = w.dk2 + align256(big * 4);
+  w.D1 = w.D2 + align256(p.rows * 4);
+  w.total = w.D1 + align256(p.rows * 4);
+  return w;
+}
+
+// ---------------------------------------------------------------- tensor maps
+
+// 5-D map over a [rows, d] bf16 tensor: (d, a, b, c, token) with the problem box's
+// token strides; boxes of (64, a_n, b_sub, c_sub, 1), 128-byte swizzle.
+squad_status encode_map(CUtensorMap* m, const void* base, const Geom& g, int d, long long rows) {
+  const cuuint64_t esz = 2;
+  cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(g.a_n), cuuint64_t(g.b_n), cuuint64_t(g.c_n), cuuint64_t(rows)};
+  cuuint64_t strides[4] = {cuuint64_t(g.sA) * d * esz, cuuint64_t(g.sB) * d * esz, cuuint64_t(g.sC) * d * esz,
+                           cuuint64_t(d) * esz};
+  cuuint32_t box[5] = {64u, cuuint32_t(g.a_n), cuuint32_t(g.b_sub), cuuint32_t(g.c_sub), 1u};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(int(r));
+  return SQUAD_OK;
+}
+
+// ---------------------------------------------------------------- launches
+
+template <int D, int KT>
+squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                             const CUtensorMap& mo, const sq::FwdArgs& a, cudaStream_t st) {
+  using Lay = sq::FwdLayout<D, KT>;
+  auto kern = sq::squad_fwd_tc_kernel<D, KT>;
+  bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0][KT];
+  if (!attr) {
+    SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
+    attr = true;
+  }
+  const int grid = a.total_probs < ds->sms ? a.total_probs : ds->sms;
+  kern<<<grid, sq::kFwdThreads, Lay::ALLOC, st>>>(mq, mk, mv, mo, a);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
+squad_status launch_fwd_tc(DeviceState* ds, int d, const Geom& g, const void* q, const void* k, const void* val,
+                           void* out, float* lse, long long rows, float scale, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mo;
+  squad_status s;
+  if ((s = encode_map(&mq, q, g, d, rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&mk, k, g, d, rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&mv, val, g, d, rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&mo, out, g, d, rows)) != SQUAD_OK) return s;
+  sq::FwdArgs a{};
+  a.g = g;
+  a.total_probs = g.bh * g.probs;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.err = ds->err;
+  a.timeout_ns = kWaitTimeoutNs;
+  const bool kt2 = g.nt >= 2;
+  if (d == 128) return kt2 ? launch_fwd_tc_t<128, 2>(ds, mq, mk, mv, mo, a, st)
+                           : launch_fwd_tc_t<128, 1>(ds, mq, mk, mv, mo, a, st);
+  return kt2 ? launch_fwd_tc_t<64, 2>(ds, mq, mk, mv, mo, a, st) : launch_fwd_tc_t<64, 1>(ds, mq, mk, mv, mo, a, st);
+}
+
+dim3 simt_grid(const Geom& g) { return dim3(unsigned(g.bh * g.probs), unsigned(sq::ceil_div(g.L, sq::kSimtWarps))); }
+
+template <typename T, int DPL>
+squad_status simt_fwd_t(const Geom& g, const void* q, const void* k, const void* val, void* out, float* lse, int d,
+                        float scale, cudaStream_t st) {
+  sq::simt_fwd_kernel<T, DPL><<<simt_grid(g), sq::kSimtWarps * 32, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(val), static_cast<T*>(out), lse, g,
+      d, scale);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
+template <typename T>
+squad_status simt_fwd(const Geom& g, const void* q, const void* k, const void* val, void* out, float* lse, int d,
+                      float scale, cudaStream_t st) {
+  switch (d / 32) {
+    case 1: return simt_fwd_t<T, 1>(g, q, k, val, out, lse, d, scale, st);
+    case 2: return simt_fwd_t<T, 2>(g, q, k, val, out, lse, d, scale, st);
+    case 3: return simt_fwd_t<T, 3>(g, q, k, val, out, lse, d, scale, st);
+    case 4: return simt_fwd_t<T, 4>(g, q, k, val, out, lse, d, scale, st);
+    case 5: return simt_fwd_t<T, 5>(g, q, k, val, out, lse, d, scale, st);
+    case 6: return simt_fwd_t<T, 6>(g, q, k, val, out, lse, d, scale, st);
+    case 7: return simt_fwd_t<T, 7>(g, q, k, val, out, lse, d, scale, st);
+    case 8: return simt_fwd_t<T, 8>(g, q, k, val, out, lse, d, scale, st);
+  }
+  return SQUAD_ERR_UNSUPPORTED;
+}
+
+// Backward of one pass on the CUDA cores: D = rowdot(dout, out); dq; dk and dval.
+template <typename T, typename TOQ, typename TOK, typename TOV, int DPL>
+squad_status simt_pass_bwd_t(const Geom& g, long long rows, const T* q, const T* k, const T* val, const T* out,
+                             const T* dout, const float* lse, float* Drow, const float* dq_add, TOQ* dq,
+                             const float* dk_add, TOK* dk, TOV* dval, int d, float scale, cudaStream_t st) {
+  const unsigned rblocks = unsigned((rows + sq::kSimtWarps - 1) / sq::kSimtWarps);
+  sq::simt_rowdot_kernel<T, DPL><<<rblocks, sq::kSimtWarps * 32, 0, st>>>(dout, out, Drow, rows, d);
+  SQ_CUDA(cudaGetLastError());
+  sq::simt_bwd_dq_kernel<T, TOQ, DPL>
+      <<<simt_grid(g), sq::kSimtWarps * 32, 0, st>>>(q, k, val, dout, lse, Drow, dq_add, dq, g, d, scale);
+  SQ_CUDA(cudaGetLastError());
+  sq::simt_bwd_dkdv_kernel<T, TOK, TOV, DPL>
+      <<<simt_grid(g), sq::kSimtWarps * 32, 0, st>>>(q, k, val, dout, lse, Drow, dk_add, dk, dval, g, d, scale);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
+template <typename T, int DPL>
+squad_status simt_bwd_t(const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k, const void* v,
+                        const void* o, const void* o1, const float* lse1, const float* lse2, const void* dout,
+                        void* dq, void* dk, void* dv, int d, cudaStream_t st) {
+  const T* Q = static_cast<const T*>(q);
+  const T* K = static_cast<const T*>(k);
+  T* dO1 = reinterpret_cast<T*>(ws + w.do1);
+  float* dQ2 = reinterpret_cast<float*>(ws + w.dq2);
+  float* dK2 = reinterpret_cast<float*>(ws + w.dk2);
+  float* D2 = reinterpret_cast<float*>(ws + w.D2);
+  float* D1 = reinterpret_cast<float*>(ws + w.D1);
+  squad_status s;
+  // global pass: values O1, upstream dout -> dQ2, dK2 (fp32) and dO1
+  s = simt_pass_bwd_t<T, float, float, T, DPL>(p.g2, p.rows, Q, K, static_cast<const T*>(o1),
+                                               static_cast<const T*>(o), static_cast<const T*>(dout), lse2, D2,
+                                               nullptr, dQ2, nullptr, dK2, dO1, d, p.scale, st);
+  if (s != SQUAD_OK) return s;
+  // local pass: values V, upstream dO1 -> dq = dq1 + dQ2, dk = dk1 + dK2, dv
+  return simt_pass_bwd_t<T, T, T, T, DPL>(p.g1, p.rows, Q, K, static_cast<const T*>(v), static_cast<const T*>(o1),
+                                          dO1, lse1, D1, dQ2, static_cast<T*>(dq), dK2, static_cast<T*>(dk),
+                                          static_cast<T*>(dv), d, p.scale, st);
+}
+
+template <typename T>
+squad_status simt_bwd(const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k, const void* v,
+                      const void* o, const void* o1, const float* lse1, const float* lse2, const void* dout, void* dq,
+                      void* dk, void* dv, int d, cudaStream_t st) {
+  switch (d / 32) {
+    case 1: return simt_bwd_t<T, 1>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 2: return simt_bwd_t<T, 2>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 3: return simt_bwd_t<T, 3>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 4: return simt_bwd_t<T, 4>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 5: return simt_bwd_t<T, 5>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 6: return simt_bwd_t<T, 6>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 7: return simt_bwd_t<T, 7>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+    case 8: return simt_bwd_t<T, 8>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, d, st);
+  }
+  return SQUAD_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+squad_status squad_attn_workspace_size(const squad_desc* desc, int which, size_t* bytes) {
+  if (bytes == nullptr) return SQUAD_ERR_INVALID_ARG;
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (which == 0) {
+    *bytes = fwd_workspace(p, desc);
+  } else if (which == 1) {
+    *bytes = bwd_workspace(p, desc).total;
+  } else {
+    return SQUAD_ERR_INVALID_ARG;
+  }
+  return SQUAD_OK;
+}
+
+squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k, const void* v, void* o, void* o1,
+                            float* lse1, float* lse2, void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SQUAD_ERR_INVALID_ARG;
+  void* o1buf = o1;
+  if (o1buf == nullptr) {
+    if (workspace == nullptr || workspace_bytes < fwd_workspace(p, desc)) return SQUAD_ERR_WORKSPACE;
+    o1buf = workspace;
+  }
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(o1buf),
+                          static_cast<const void*>(lse1), static_cast<const void*>(lse2)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int d = desc->d;
+  if (desc->dtype == SQUAD_BF16) {
+    if ((s = launch_fwd_tc(ds, d, p.g1, q, k, v, o1buf, lse1, p.rows, p.scale, st)) != SQUAD_OK) return s;
+    return launch_fwd_tc(ds, d, p.g2, q, k, o1buf, o, lse2, p.rows, p.scale, st);
+  }
+  if ((s = simt_fwd<float>(p.g1, q, k, v, o1buf, lse1, d, p.scale, st)) != SQUAD_OK) return s;
+  return simt_fwd<float>(p.g2, q, k, o1buf, o, lse2, d, p.scale, st);
+}
+
+squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* q, const void* k,
+                                 const void* val, void* out, float* lse, void* stream) {
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (stage != 1 && stage != 2) return SQUAD_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || val == nullptr || out == nullptr) return SQUAD_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, val, static_cast<const void*>(out), static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Geom& g = stage == 1 ? p.g1 : p.g2;
+  if (desc->dtype == SQUAD_BF16) return launch_fwd_tc(ds, desc->d, g, q, k, val, out, lse, p.rows, p.scale, st);
+  return simt_fwd<float>(g, q, k, val, out, lse, desc->d, p.scale, st);
+}
+
+squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                            const void* o1, const float* lse1, const float* lse2, const void* dout, void* dq,
+                            void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  for (const void* ptr : {q, k, v, o, o1, static_cast<const void*>(lse1), static_cast<const void*>(lse2), dout,
+                          static_cast<const void*>(dq), static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (ptr == nullptr) return SQUAD_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, o1, static_cast<const void*>(lse1), static_cast<const void*>(lse2), dout,
+                          static_cast<const void*>(dq), static_cast<const void*>(dk), static_cast<const void*>(dv),
+                          static_cast<const void*>(workspace)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  const BwdWs w = bwd_workspace(p, desc);
+  if (workspace == nullptr || workspace_bytes < w.total) return SQUAD_ERR_WORKSPACE;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (desc->dtype == SQUAD_BF16)
+    return simt_bwd<__nv_bfloat16>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, desc->d, st);
+  return simt_bwd<float>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, desc->d, st);
+}
+
+squad_status squad_plan_info(const squad_desc* desc, int stage, int* info) {
+  if (info == nullptr || (stage != 1 && stage != 2)) return SQUAD_ERR_INVALID_ARG;
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  Geom g = stage == 1 ? p.g1 : p.g2;
+  if (desc->dtype != SQUAD_BF16 && !sq::plan_tiles(g)) return SQUAD_ERR_UNSUPPORTED;
+  info[0] = g.L;
+  info[1] = g.probs;
+  info[2] = g.nt;
+  info[3] = g.box_rows;
+  info[4] = g.a_n;
+  info[5] = g.b_sub;
+  info[6] = g.c_sub;
+  info[7] = g.nt >= 2 ? 2 : 1;
+  return SQUAD_OK;
+}
+
+squad_status squad_poll_device_error(void* stream) {
+  SQ_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  SQ_CUDA(cudaMemcpyFromSymbol(&v, g_squad_dev_err, sizeof(int)));
+  if (v != 0) {
+    const int zero = 0;
+    SQ_CUDA(cudaMemcpyToSymbol(g_squad_dev_err, &zero, sizeof(int)));
+    return SQUAD_ERR_TIMEOUT;
+  }
+  return SQUAD_OK;
+}
+
+const char* squad_strerror(int status) {
+  switch (status) {
+    case SQUAD_OK: return "ok";
+    case SQUAD_ERR_INVALID_ARG: return "invalid argument";
+    case SQUAD_ERR_SHAPE: return "invalid shape";
+    case SQUAD_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case SQUAD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SQUAD_ERR_CUDA: return "CUDA error";
+    case SQUAD_ERR_TIMEOUT: return "device wait timed out";
+    case SQUAD_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int squad_last_cuda_error(void) { return t_last_cuda; }
+
+int squad_version(void) { return kVersion; }
+
+}  // extern "C"

@@ -1,0 +1,135 @@
+"""Host-side checks of the C ABI (no GPU needed): exports, argument checks, plans.
+
+Every check here returns before the library makes any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sub_quadratic_two_b200 as sq
+from sub_quadratic_two_b200 import SquadDesc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "squad.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA, TIMEOUT, WORKSPACE = range(8)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return sq.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(squad_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "squad_attn_fwd" in names and "squad_attn_bwd" in names
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_version_and_strerror(lib):
+    assert lib.squad_version() >= 10000
+    for code in range(8):
+        assert lib.squad_strerror(code)
+    assert lib.squad_strerror(99) == b"unknown status"
+
+
+def _desc(**kw):
+    base = dict(B=1, heads=2, d=128, T=4, H=8, W=8, tT=1, tH=4, tW=4, dtype=sq.SQUAD_BF16, scale=0.0)
+    base.update(kw)
+    return SquadDesc(**base)
+
+
+FAKE = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: calls fail before any launch
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def _fwd(lib, desc, q=FAKE, k=FAKE, v=FAKE, o=FAKE, o1=FAKE, ws=None, ws_bytes=0):
+    return lib.squad_attn_fwd(ctypes.byref(desc), q, k, v, o, o1, None, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(tH=3), SHAPE),              # 3 does not divide H=8
+    (dict(T=0), SHAPE),
+    (dict(tW=-1), SHAPE),
+    (dict(dtype=7), INVALID),
+    (dict(d=96), UNSUPPORTED),        # bf16 kernels take d in {64, 128}
+    (dict(W=256, tW=1), UNSUPPORTED), # a global-pass box row of 256 > 128 tokens
+    (dict(dtype=sq.SQUAD_F32, d=48), UNSUPPORTED),
+    (dict(B=40000, heads=64, T=32, H=32, W=32, tT=1, tH=1, tW=32), SHAPE),  # rows >= 2^31
+])
+def test_shape_and_type_errors(lib, kw, code):
+    assert _fwd(lib, _desc(**kw)) == code
+
+
+def test_null_and_alignment_errors(lib):
+    d = _desc()
+    assert lib.squad_attn_fwd(None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 0, None) == INVALID
+    assert _fwd(lib, d, q=None) == INVALID
+    assert _fwd(lib, d, k=MISALIGNED) == ALIGN
+    assert _fwd(lib, d, o=MISALIGNED) == ALIGN
+    # o1 == NULL needs the workspace
+    assert _fwd(lib, d, o1=None) == WORKSPACE
+    need = sq.workspace_size(d, 0)
+    assert _fwd(lib, d, o1=None, ws=FAKE, ws_bytes=need - 1) == WORKSPACE
+
+
+def test_backward_argument_errors(lib):
+    d = _desc()
+    args = [FAKE] * 11
+    need = sq.workspace_size(d, 1)
+    assert lib.squad_attn_bwd(ctypes.byref(d), *args, FAKE, need - 16, None) == WORKSPACE
+    args2 = list(args)
+    args2[3] = None  # o
+    assert lib.squad_attn_bwd(ctypes.byref(d), *args2, FAKE, need, None) == INVALID
+    args3 = list(args)
+    args3[8] = MISALIGNED  # dq
+    assert lib.squad_attn_bwd(ctypes.byref(d), *args3, FAKE, need, None) == ALIGN
+
+
+def test_workspace_sizes(lib):
+    d = _desc()
+    rows = 1 * 2 * 256
+    assert sq.workspace_size(d, 0) == rows * 128 * 2
+    # dO1 (bf16) + dQ2, dK2 (fp32) + two fp32 row vectors, each 256-byte aligned
+    assert sq.workspace_size(d, 1) == rows * 128 * 2 + 2 * rows * 128 * 4 + 2 * rows * 4
+    with pytest.raises(sq.SquadError):
+        sq.workspace_size(d, 5)
+
+
+def _plan(lib, desc, stage):
+    info = (ctypes.c_int * 8)()
+    assert lib.squad_plan_info(ctypes.byref(desc), stage, info) == OK
+    return list(info)
+
+
+@pytest.mark.parametrize("grid,tile,expect1,expect2", [
+    # local pass of the 5B shape: 220-token windows cut into 120 + 100 token boxes (6 and 5 rows of 20)
+    ((31, 22, 40), (1, 11, 20), [220, 124, 2, 120, 20, 6, 1, 2], [124, 220, 1, 124, 2, 2, 31, 1]),
+    # long video: 440-token windows -> 4 boxes of 6 rows (online softmax over 2 groups)
+    ((61, 22, 40), (1, 22, 20), [440, 122, 4, 120, 20, 6, 1, 2], [122, 440, 1, 122, 2, 1, 61, 1]),
+    ((8, 16, 16), (2, 4, 8), [64, 32, 1, 64, 8, 4, 2, 1], [32, 64, 1, 32, 2, 4, 4, 1]),
+    ((4, 8, 8), (1, 4, 4), [16, 16, 1, 16, 4, 4, 1, 1], [16, 16, 1, 16, 2, 2, 4, 1]),
+])
+def test_plans_of_the_workloads(lib, grid, tile, expect1, expect2):
+    d = _desc(B=1, heads=24, T=grid[0], H=grid[1], W=grid[2], tT=tile[0], tH=tile[1], tW=tile[2])
+    assert _plan(lib, d, 1) == expect1
+    assert _plan(lib, d, 2) == expect2
+
+
+def test_plan_tiles_cover_problem(lib):
+    # every tiling covers the problem exactly: nt boxes, the last one ragged
+    for grid, tile in [((6, 10, 12), (3, 5, 12)), ((2, 40, 30), (1, 20, 15)), ((9, 4, 4), (1, 2, 2))]:
+        d = _desc(T=grid[0], H=grid[1], W=grid[2], tT=tile[0], tH=tile[1], tW=tile[2])
+        for stage in (1, 2):
+            L, probs, nt, box, a, b, c, kt = _plan(lib, d, stage)
+            assert box == a * b * c <= 128
+            assert (nt - 1) * box < L <= nt * box

@@ -1,0 +1,210 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (stated for the operator's workloads):
+  fp32 path      : max |err| <= 1e-5 on O, O1, LSE and on dQ, dK, dV;
+  bf16 forward   : max |err| <= 1.5e-2 and mean |err| <= 2e-3 on O and O1,
+                   max |err| <= 2e-3 on LSE (fp32 scores of bf16 inputs);
+  bf16 gradients : max |err| <= 3e-2 on dQ, dK, dV.
+Both sides read the same seeded inputs (bf16 values widened to fp64 for the
+oracle). Full-size workloads run the GPU on every head and compare whole
+(batch, head) slices, which are independent problems, against the oracle run
+on those slices alone.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sub_quadratic_two_b200 as sq
+from workloads import WORKLOADS, make_inputs, random_problem
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+BF16_MAX, BF16_MEAN, LSE_TOL, GRAD_MAX = 1.5e-2, 2e-3, 2e-3, 3e-2
+
+
+def _dev(*ts):
+    return [t.contiguous().cuda() for t in ts]
+
+
+def gpu_fwd(q, k, v, grid, tile, scale=None):
+    qd, kd, vd = _dev(q, k, v)
+    o, o1, l1, l2 = sq.squad_attn_fwd(qd, kd, vd, grid, tile, scale)
+    sq.poll_device_error()
+    return [x.cpu().double().numpy() for x in (o, o1, l1, l2)]
+
+
+def gpu_bwd(q, k, v, do, grid, tile, scale=None):
+    qd, kd, vd, dod = _dev(q, k, v, do)
+    o, o1, l1, l2 = sq.squad_attn_fwd(qd, kd, vd, grid, tile, scale)
+    dq, dk, dv = sq.squad_attn_bwd(qd, kd, vd, o, o1, l1, l2, dod, grid, tile, scale)
+    sq.poll_device_error()
+    return [x.cpu().double().numpy() for x in (dq, dk, dv)]
+
+
+def _err(a, b):
+    e = np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))
+    return float(e.max()), float(e.mean())
+
+
+def assert_bf16_fwd(got, ref, what):
+    mx, mean = _err(got, ref)
+    assert np.isfinite(got).all(), what
+    assert mx <= BF16_MAX and mean <= BF16_MEAN, f"{what}: max {mx:.3e} mean {mean:.3e}"
+
+
+def assert_close(got, ref, tol, what):
+    mx, _ = _err(got, ref)
+    assert np.isfinite(got).all(), what
+    assert mx <= tol, f"{what}: max {mx:.3e} > {tol:.1e}"
+
+
+def check_fwd_bf16(inp, grid, tile, heads=None):
+    o, o1, l1, l2 = gpu_fwd(inp.q, inp.k, inp.v, grid, tile)
+    sel = (slice(None), slice(None)) if heads is None else (slice(0, 1), heads)
+    ro, ro1, rl1, rl2, _ = oracle.squad_fwd(inp.q[sel], inp.k[sel], inp.v[sel], grid, tile)
+    assert_bf16_fwd(o1[sel], ro1, "O1")
+    assert_bf16_fwd(o[sel], ro, "O")
+    assert_close(l1[sel], rl1, LSE_TOL, "LSE1")
+    assert_close(l2[sel], rl2, LSE_TOL, "LSE2")
+
+
+# ------------------------------------------------------------------ fp32 path (CUDA cores)
+
+def test_tiny_fp32_forward(cuda_ok):
+    wl = WORKLOADS["tiny_fp32"]
+    inp = make_inputs(wl)
+    o, o1, l1, l2 = gpu_fwd(inp.q, inp.k, inp.v, wl.grid, wl.tile)
+    ro, ro1, rl1, rl2, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, wl.grid, wl.tile)
+    assert_close(o, ro, F32_TOL, "O")
+    assert_close(o1, ro1, F32_TOL, "O1")
+    assert_close(l1, rl1, F32_TOL, "LSE1")
+    assert_close(l2, rl2, F32_TOL, "LSE2")
+
+
+def test_tiny_fp32_backward(cuda_ok):
+    wl = WORKLOADS["tiny_fp32"]
+    inp = make_inputs(wl)
+    do = torch.randn(inp.q.shape, generator=torch.Generator().manual_seed(101))
+    got = gpu_bwd(inp.q, inp.k, inp.v, do, wl.grid, wl.tile)
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, do, wl.grid, wl.tile)
+    for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
+        assert_close(a, b, F32_TOL, name)
+
+
+@pytest.mark.parametrize("grid,tile,d", [((3, 6, 10), (3, 2, 5), 32), ((2, 4, 6), (2, 4, 6), 96), ((5, 2, 3), (1, 1, 1), 64)])
+def test_fp32_other_shapes(cuda_ok, grid, tile, d):
+    inp = random_problem(7, 2, 2, d, grid, tile, dtype=torch.float32, with_do=True)
+    o, o1, _, _ = gpu_fwd(inp.q, inp.k, inp.v, grid, tile)
+    ro, ro1, _, _, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, grid, tile)
+    assert_close(o, ro, F32_TOL, "O")
+    assert_close(o1, ro1, F32_TOL, "O1")
+    got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
+        assert_close(a, b, F32_TOL, name)
+
+
+# ------------------------------------------------------------------ bf16 forward (tensor cores)
+
+def test_small_bf16_forward(cuda_ok):
+    wl = WORKLOADS["small_bf16"]
+    check_fwd_bf16(make_inputs(wl), wl.grid, wl.tile)
+
+
+@pytest.mark.parametrize("grid,tile,heads,d", [
+    ((4, 22, 40), (1, 11, 20), 2, 128),   # 220-token windows: two boxes, ragged 100-token tail
+    ((2, 44, 40), (1, 22, 20), 2, 128),   # 440-token windows: four boxes, online softmax over two groups
+    ((40, 8, 8), (1, 2, 2), 1, 128),      # 640-token groups in the global pass: five boxes, three groups
+    ((6, 12, 16), (2, 6, 8), 2, 64),      # tT > 1, d = 64
+    ((3, 5, 7), (3, 5, 7), 2, 128),       # one window: the global pass has one token
+    ((2, 6, 10), (1, 1, 1), 1, 128),      # one-token windows: the local pass is the identity
+    ((9, 6, 6), (3, 2, 3), 3, 128),       # odd sizes everywhere
+])
+def test_bf16_forward_shapes(cuda_ok, grid, tile, heads, d):
+    inp = random_problem(17, 1, heads, d, grid, tile, dtype=torch.bfloat16, k_bias_std=1.0)
+    check_fwd_bf16(inp, grid, tile)
+
+
+def test_bf16_forward_batch_and_explicit_scale(cuda_ok):
+    grid, tile = (4, 8, 8), (2, 4, 4)
+    inp = random_problem(19, 3, 2, 128, grid, tile, dtype=torch.bfloat16)
+    o, o1, _, _ = gpu_fwd(inp.q, inp.k, inp.v, grid, tile, scale=0.05)
+    ro, ro1, _, _, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, grid, tile, scale=0.05)
+    assert_bf16_fwd(o, ro, "O")
+    assert_bf16_fwd(o1, ro1, "O1")
+
+
+def test_bf16_forward_deterministic(cuda_ok):
+    wl = WORKLOADS["small_bf16"]
+    inp = make_inputs(wl)
+    a = gpu_fwd(inp.q, inp.k, inp.v, wl.grid, wl.tile)
+    b = gpu_fwd(inp.q, inp.k, inp.v, wl.grid, wl.tile)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_wan5b_forward_full_size(cuda_ok):
+    wl = WORKLOADS["wan5b_fwd"]
+    inp = make_inputs(wl)
+    check_fwd_bf16(inp, wl.grid, wl.tile, heads=[0, 13, 23])
+
+
+def test_long_video_forward_full_size(cuda_ok):
+    wl = WORKLOADS["long_video"]
+    inp = make_inputs(wl)
+    check_fwd_bf16(inp, wl.grid, wl.tile, heads=[7])
+
+
+# ------------------------------------------------------------------ bf16 backward
+
+@pytest.mark.parametrize("grid,tile,heads", [((4, 8, 8), (1, 4, 4), 2), ((4, 22, 40), (1, 11, 20), 1)])
+def test_bf16_backward_shapes(cuda_ok, grid, tile, heads):
+    inp = random_problem(23, 1, heads, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
+        assert_close(a, b, GRAD_MAX, name)
+
+
+def test_wan5b_training_step_full_size(cuda_ok):
+    wl = WORKLOADS["wan5b_train"]
+    inp = make_inputs(wl)
+    got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, wl.grid, wl.tile)
+    for b, h in [(0, 3), (1, 20)]:
+        sel = (slice(b, b + 1), slice(h, h + 1))
+        ref = oracle.squad_bwd(inp.q[sel], inp.k[sel], inp.v[sel], inp.do[sel], wl.grid, wl.tile)
+        for name, a, r in zip(("dQ", "dK", "dV"), got, ref):
+            assert_close(a[sel], r, GRAD_MAX, f"{name}[b={b},h={h}]")
+
+
+def test_autograd_function(cuda_ok):
+    grid, tile = (4, 8, 8), (1, 4, 4)
+    inp = random_problem(29, 1, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    q, k, v = (x.cuda().requires_grad_(True) for x in (inp.q, inp.k, inp.v))
+    o = sq.attention(q, k, v, grid, tile)
+    o.backward(inp.do.cuda())
+    ref_o, *_ = oracle.squad_fwd(inp.q, inp.k, inp.v, grid, tile)
+    assert_bf16_fwd(o.detach().cpu().double().numpy(), ref_o, "O")
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, t, r in zip(("dQ", "dK", "dV"), (q, k, v), ref):
+        assert_close(t.grad.cpu().double().numpy(), r, GRAD_MAX, name)
+
+
+def test_inference_forward_uses_workspace(cuda_ok):
+    wl = WORKLOADS["small_bf16"]
+    inp = make_inputs(wl)
+    qd, kd, vd = _dev(inp.q, inp.k, inp.v)
+    o_save, *_ = sq.squad_attn_fwd(qd, kd, vd, wl.grid, wl.tile, save=True)
+    o_inf, o1, l1, l2 = sq.squad_attn_fwd(qd, kd, vd, wl.grid, wl.tile, save=False)
+    sq.poll_device_error()
+    assert o1 is None and l1 is None
+    assert torch.equal(o_save, o_inf)
+
+
+def test_cpu_tensors_are_rejected():
+    grid, tile = (2, 4, 4), (1, 2, 2)
+    inp = random_problem(31, 1, 1, 64, grid, tile, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sq.squad_attn_fwd(inp.q, inp.k, inp.v, grid, tile)

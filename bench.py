@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the SQuad-Attention hot path on B200.
+
+Headline: forward ms and TFLOP/s at 27,280 tokens (the Wan 2.2 5B DiT attention
+shape: B=1, 24 heads, d=128, grid 31x22x40, 1x11x20 windows), bf16 in / fp32
+accumulate, as a fraction of the measured bf16 tensor-core peak. One step is one
+forward (local pass, then global pass) over one batch of synthetic inputs that
+are resident in HBM. The data are synthetic (seeded N(0,1) draws shaped like the
+workload; the pages' videos and weights are not available).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs the full workload on its
+own GPU (independent (batch, head) problems: weak scaling, no data-path
+collective); the timed region is bracketed by barriers and the slowest rank's
+time is reported. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SQuad-attn fwd ms & TFLOP/s at 27,280 tokens; % of B200 bf16 TC peak"
+HEADLINE = "wan5b_fwd"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training-step leg")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget for the CPU baseline")
+    ap.add_argument("--profile", action="store_true",
+                    help="profiling driver: one warm-up forward, then one forward (two kernel launches), no timing")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks (NVML, read-only)
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons every ~5 ms on one GPU (read-only NVML)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not fail the bench
+            self.err = str(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons(self):
+        nv = self.nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return getattr(nv, fn)(self.h)
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                self.samples.append((time.perf_counter(), mhz, self._reasons()))
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": f"NVML unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "nvml, 5 ms, inside the timed region"
+        if not win:  # region shorter than the sampling interval: take the nearest samples
+            win = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+            note = "nvml, nearest samples to a short timed region"
+        mask = 0
+        for s in win:
+            mask |= s[2]
+        reasons = [k for k, v in self.REASONS.items() if mask & v and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in win) if win else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(win), "note": note}
+
+
+# ------------------------------------------------------------------ helpers
+
+def source_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def read_traffic(kernel_key: str, src_path: str, units_scale: float = 1.0):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, or None when the
+    summary is missing or was taken on a different version of the kernel source."""
+    prof = os.path.join(ROOT, "profiles", "ncu_fwd_tc_wan5b.md")
+    if not os.path.exists(prof):
+        return None
+    text = open(prof).read()
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_val = re.search(rf"{kernel_key}_dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_val or m_sha.group(1) != source_sha(src_path):
+        return None
+    return int(m_val.group(1)) * units_scale
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl, budget_s: float, threads: int):
+    """The fp64 oracle, as it stands, over whole heads of the workload until the budget is spent."""
+    import oracle
+    from workloads import make_inputs
+    inp = make_inputs(wl)
+    flops, secs, heads = 0.0, 0.0, 0
+    per_head = 4.0 * wl.n * wl.d * (wl.w + wl.m)
+    for h in range(wl.heads):
+        sel = (slice(0, 1), slice(h, h + 1))
+        t = time.perf_counter()
+        oracle.squad_fwd(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, wl.tile, threads=threads)
+        secs += time.perf_counter() - t
+        flops += per_head
+        heads += 1
+        if secs >= budget_s:
+            break
+    return flops, secs, heads
+
+
+# ------------------------------------------------------------------ reference arm (the oracle)
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0  # the oracle arm runs on rank 0 only
+    from workloads import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    cores = cpu_cores()
+    import oracle
+    from workloads import make_inputs
+    inp = make_inputs(wl)
+    sel = (slice(0, 1), slice(0, 1))   # each step: one (batch, head) slice of the workload
+    per_step = 4.0 * wl.n * wl.d * (wl.w + wl.m)
+    for _ in range(args.warmup):
+        oracle.squad_fwd(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, wl.tile, threads=cores)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.squad_fwd(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, wl.tile, threads=cores)
+        times.append(time.perf_counter() - t)
+    ms = 1e3 * sum(times) / len(times)
+    value = per_step / (ms / 1e3) / 1e12
+    sample = f"one (batch, head) slice of {wl.name} per step: n={wl.n}, d={wl.d}, w={wl.w}, m={wl.m}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample": "1 of %d heads" % wl.heads, "grid": list(wl.grid),
+                   "tile": list(wl.tile), "d": wl.d},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import sub_quadratic_two_b200 as sq
+    from workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    desc = sq.make_desc(q, wl.grid, wl.tile, None)
+    ws = torch.empty(sq.workspace_size(desc, 0), device=dev, dtype=torch.uint8)
+    flush = None if args.profile else torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    flops = wl.fwd_flops()
+
+    def step():
+        sq.squad_attn_fwd(q, k, v, wl.grid, wl.tile, save=False, out=o, workspace=ws)
+
+    if args.profile:
+        step()
+        torch.cuda.synchronize()
+        step()
+        sq.poll_device_error()
+        print("profile run done")
+        return 0
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    sq.poll_device_error()
+
+    # ---------------- timed region: exactly K steps, L2 flushed before each, device events per step
+    sampler = ClockSampler(local)
+    sampler.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    barrier()
+    sampler.stop()
+    sq.poll_device_error()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms))
+    ms_per_step = total_ms / args.steps
+    value = world * flops / (ms_per_step / 1e3) / 1e12
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    # ---------------- per-pass kernel timing (same stream, events, L2 flushed)
+    o1 = torch.empty_like(q)
+    lse = None
+    reps = max(10, min(args.steps, 50))
+    pass_ms = {}
+    for stage in (1, 2):
+        val = v if stage == 1 else o1
+        out = o1 if stage == 1 else o
+        sq.squad_attn_fwd_pass(stage, q, k, val, out, wl.grid, wl.tile, lse=lse)
+        evs = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            sq.squad_attn_fwd_pass(stage, q, k, val, out, wl.grid, wl.tile, lse=lse)
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        pass_ms[stage] = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    sq.poll_device_error()
+    rows = wl.B * wl.heads * wl.n
+    pass_bytes = 4 * rows * wl.d * 2   # each pass reads 3 [rows, d] bf16 tensors and writes one
+    pass_flops = {1: 4.0 * rows * wl.d * wl.w, 2: 4.0 * rows * wl.d * wl.m}
+    dom = max(pass_ms, key=pass_ms.get)
+    achieved = pass_bytes / (pass_ms[dom] / 1e3) / 1e9
+    src = os.path.join(ROOT, "sub_quadratic_two_b200", "csrc", "squad_fwd_tc.cuh")
+    roofline = {
+        "bound": "hbm", "kernel": f"squad_fwd_tc_kernel (pass {dom})", "achieved": achieved,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+        "traffic": read_traffic(f"pass{dom}", src), "algorithmic_bytes_per_launch": pass_bytes,
+        "peak_source": f"{peak_src} hbm_gbs (burst, kernel timed alone)",
+    }
+    passes = {f"pass{s}": {"ms": pass_ms[s], "GB/s": pass_bytes / (pass_ms[s] / 1e3) / 1e9,
+                           "TFLOP/s": pass_flops[s] / (pass_ms[s] / 1e3) / 1e12} for s in (1, 2)}
+
+    # ---------------- end to end through the public API, host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.pin_memory() for t in (inp.q, inp.k, inp.v))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        ek = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            dq_, dk_, dv_ = (t.to(dev, non_blocking=True) for t in (hq, hk, hv))
+            out_ = sq.attention(dq_, dk_, dv_, wl.grid, wl.tile)
+            ho.copy_(out_, non_blocking=True)
+
+        with torch.no_grad():
+            for _ in range(2):
+                e2e_step()
+            barrier()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(ek):
+                e2e_step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b)) / ek
+        e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": ek,
+               "path": "sub_quadratic_two_b200.attention on pinned host tensors"}
+
+    # ---------------- training step (forward + backward), the distillation workload
+    train = None
+    if not args.no_train:
+        twl = WORKLOADS["wan5b_train"]
+        tin = make_inputs(twl)
+        tq, tk, tv, tdo = (t.to(dev) for t in (tin.q, tin.k, tin.v, tin.do))
+        del tin
+
+        def train_step():
+            o_, o1_, l1_, l2_ = sq.squad_attn_fwd(tq, tk, tv, twl.grid, twl.tile, save=True)
+            sq.squad_attn_bwd(tq, tk, tv, o_, o1_, l1_, l2_, tdo, twl.grid, twl.tile)
+
+        for _ in range(2):
+            train_step()
+        tsteps = 5
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(tsteps):
+            train_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        sq.poll_device_error()
+        tms = max_over_ranks(a.elapsed_time(b)) / tsteps
+        tfl = twl.fwd_flops() + twl.bwd_flops()
+        train = {"workload": twl.name, "ms_per_step": tms, "TFLOP/s": world * tfl / (tms / 1e3) / 1e12,
+                 "useful_flops_per_step": tfl, "steps": tsteps,
+                 "note": "backward runs on CUDA-core kernels in this version"}
+        del tq, tk, tv, tdo
+
+    # ---------------- CPU baseline: the oracle on host cores, rank 0 at N=1 only
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = cpu_cores()
+        fl, secs, heads = oracle_sample(wl, args.cpu_seconds, cores)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"{heads} of {wl.heads} heads of {wl.name} (fp64, {secs:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
+                       "grid": list(wl.grid), "tile": list(wl.tile), "w": wl.w, "m": wl.m,
+                       "useful_flops_per_step": flops,
+                       "l2": "flushed (512 MiB write) before every timed step; inputs 503 MB > L2",
+                       "parallelism": f"replicas x{world} (independent problems per GPU)"},
+            "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
+                                  "measured_sustained": value / world / peaks.get("bf16_tflops_sustained", 1),
+                                  "spec_dense_2250": value / world / 2250.0, "source": peak_src},
+            "roofline": roofline, "passes": passes, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * args.steps, "clocks": clocks, "train_step": train,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

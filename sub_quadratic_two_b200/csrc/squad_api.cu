@@ -14,6 +14,7 @@
 
 #include "squad.h"
 #include "geometry.h"
+#include "squad_bwd_tc.cuh"
 #include "squad_fwd_tc.cuh"
 #include "squad_simt.cuh"
 
@@ -47,6 +48,7 @@ struct DeviceState {
   int sms = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
   bool fwd_attr_set[2][3] = {};  // [D=64/128][KT]
+  bool bwd_attr_set[2][2][2] = {};  // [D=64/128][mode][out_f32]
 };
 
 std::mutex g_mu;
@@ -264,6 +266,91 @@ squad_status simt_bwd_t(const Plan& p, const BwdWs& w, uint8_t* ws, const void* 
                                           static_cast<T*>(dv), d, p.scale, st);
 }
 
+// ---------------- tensor-core backward (bf16)
+
+template <int D, int MODE, bool F32>
+squad_status launch_bwd_tc_t(DeviceState* ds, const CUtensorMap* maps, const sq::BwdArgs& a, cudaStream_t st) {
+  using Lay = sq::BwdLayout<D>;
+  auto kern = sq::squad_bwd_tc_kernel<D, MODE, F32>;
+  bool& attr = ds->bwd_attr_set[D == 128 ? 1 : 0][MODE][F32 ? 1 : 0];
+  if (!attr) {
+    SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
+    attr = true;
+  }
+  const int grid = a.total_items < ds->sms ? a.total_items : ds->sms;
+  kern<<<grid, sq::kBwdThreads, Lay::ALLOC, st>>>(maps[0], maps[1], maps[2], maps[3], a);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
+template <int MODE, bool F32>
+squad_status launch_bwd_tc(DeviceState* ds, int d, const CUtensorMap* maps, const sq::BwdArgs& a, cudaStream_t st) {
+  if (d == 128) return launch_bwd_tc_t<128, MODE, F32>(ds, maps, a, st);
+  return launch_bwd_tc_t<64, MODE, F32>(ds, maps, a, st);
+}
+
+// Backward of one pass on the tensor cores. q, k: inputs; val: the pass's values;
+// out: the pass's output; dout: its upstream gradient. f32_out selects fp32 dq/dk
+// (the global pass, whose parts are summed into the local pass's results).
+squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, const void* q, const void* k,
+                         const void* val, const void* out, const void* dout, const float* lse, float* Drow,
+                         const float* dq_add, void* dq, const float* dk_add, void* dk, __nv_bfloat16* dval,
+                         bool f32_out, cudaStream_t st) {
+  const unsigned rblocks = unsigned((p.rows + sq::kSimtWarps - 1) / sq::kSimtWarps);
+  if (d == 128)
+    sq::simt_rowdot_kernel<__nv_bfloat16, 4><<<rblocks, sq::kSimtWarps * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), Drow, p.rows, d);
+  else
+    sq::simt_rowdot_kernel<__nv_bfloat16, 2><<<rblocks, sq::kSimtWarps * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), Drow, p.rows, d);
+  SQ_CUDA(cudaGetLastError());
+  CUtensorMap maps[4];
+  squad_status s;
+  if ((s = encode_map(&maps[0], q, g, d, p.rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&maps[1], k, g, d, p.rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&maps[2], val, g, d, p.rows)) != SQUAD_OK) return s;
+  if ((s = encode_map(&maps[3], dout, g, d, p.rows)) != SQUAD_OK) return s;
+  sq::BwdArgs a{};
+  a.g = g;
+  a.total_items = g.bh * g.probs * g.nt;
+  a.scale = p.scale;
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.Drow = Drow;
+  a.err = ds->err;
+  a.timeout_ns = kWaitTimeoutNs;
+  // dq
+  a.add = dq_add;
+  a.out_main = dq;
+  a.out_val = nullptr;
+  s = f32_out ? launch_bwd_tc<sq::MODE_DQ, true>(ds, d, maps, a, st)
+              : launch_bwd_tc<sq::MODE_DQ, false>(ds, d, maps, a, st);
+  if (s != SQUAD_OK) return s;
+  // dk, dval
+  a.add = dk_add;
+  a.out_main = dk;
+  a.out_val = dval;
+  return f32_out ? launch_bwd_tc<sq::MODE_DKDV, true>(ds, d, maps, a, st)
+                 : launch_bwd_tc<sq::MODE_DKDV, false>(ds, d, maps, a, st);
+}
+
+squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k,
+                    const void* v, const void* o, const void* o1, const float* lse1, const float* lse2,
+                    const void* dout, void* dq, void* dk, void* dv, int d, cudaStream_t st) {
+  auto* dO1 = reinterpret_cast<__nv_bfloat16*>(ws + w.do1);
+  float* dQ2 = reinterpret_cast<float*>(ws + w.dq2);
+  float* dK2 = reinterpret_cast<float*>(ws + w.dk2);
+  float* D2 = reinterpret_cast<float*>(ws + w.D2);
+  float* D1 = reinterpret_cast<float*>(ws + w.D1);
+  squad_status s;
+  // global pass: values O1, output O, upstream dout -> dQ2, dK2 (fp32) and dO1
+  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, D2, nullptr, dQ2, nullptr, dK2, dO1, true, st);
+  if (s != SQUAD_OK) return s;
+  // local pass: values V, output O1, upstream dO1 -> dq = dq1 + dQ2, dk = dk1 + dK2, dv
+  return tc_pass_bwd(ds, p, d, p.g1, q, k, v, o1, dO1, lse1, D1, dQ2, dq, dK2, dk,
+                     static_cast<__nv_bfloat16*>(dv), false, st);
+}
+
 template <typename T>
 squad_status simt_bwd(const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k, const void* v,
                       const void* o, const void* o1, const float* lse1, const float* lse2, const void* dout, void* dq,
@@ -365,7 +452,7 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (desc->dtype == SQUAD_BF16)
-    return simt_bwd<__nv_bfloat16>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, desc->d, st);
+    return tc_bwd(ds, p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, desc->d, st);
   return simt_bwd<float>(p, w, ws, q, k, v, o, o1, lse1, lse2, dout, dq, dk, dv, desc->d, st);
 }
 

@@ -392,7 +392,7 @@ def main():
         tfl = twl.fwd_flops() + twl.bwd_flops()
         train = {"workload": twl.name, "ms_per_step": tms, "TFLOP/s": world * tfl / (tms / 1e3) / 1e12,
                  "useful_flops_per_step": tfl, "steps": tsteps,
-                 "note": "backward runs on CUDA-core kernels in this version"}
+                 "note": "backward: tcgen05 dq and dk/dv kernels per pass"}
         del tq, tk, tv, tdo
 
     # ---------------- CPU baseline: the oracle on host cores, rank 0 at N=1 only

@@ -159,9 +159,17 @@ def test_long_video_forward_full_size(cuda_ok):
 
 # ------------------------------------------------------------------ bf16 backward
 
-@pytest.mark.parametrize("grid,tile,heads", [((4, 8, 8), (1, 4, 4), 2), ((4, 22, 40), (1, 11, 20), 1)])
-def test_bf16_backward_shapes(cuda_ok, grid, tile, heads):
-    inp = random_problem(23, 1, heads, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+@pytest.mark.parametrize("grid,tile,heads,d", [
+    ((4, 8, 8), (1, 4, 4), 2, 128),
+    ((4, 22, 40), (1, 11, 20), 1, 128),   # ragged 220-token windows
+    ((2, 44, 40), (1, 22, 20), 1, 128),   # 440-token windows: four boxes per problem
+    ((40, 8, 8), (1, 2, 2), 1, 128),      # 640-token global groups: five boxes
+    ((6, 12, 16), (2, 6, 8), 2, 64),      # tT > 1, d = 64
+    ((3, 5, 7), (3, 5, 7), 1, 128),       # one window
+    ((2, 6, 10), (1, 1, 1), 1, 128),      # one-token windows
+])
+def test_bf16_backward_shapes(cuda_ok, grid, tile, heads, d):
+    inp = random_problem(23, 1, heads, d, grid, tile, dtype=torch.bfloat16, with_do=True)
     got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
     ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
     for name, a, b in zip(("dQ", "dK", "dV"), got, ref):

@@ -93,6 +93,32 @@ squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k
 squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* q, const void* k,
                                  const void* val, void* out, float* lse, void* stream);
 
+/* Forward that allocates nothing, not even a workspace. The paper has no
+ * counterpart: this entry point exists for callers that cannot hand the
+ * library device memory for scratch, e.g. code running inside a host
+ * framework that owns every device allocation (a fixed memory pool or arena)
+ * and forbids side allocations, or latency-critical code that must not call
+ * cudaMalloc because it may synchronise the device. Such callers pass only
+ * their inputs and outputs; the local-pass output, which squad_attn_fwd keeps
+ * in o1 or in the caller's workspace, lives here in a fixed 32 MiB array of
+ * device memory inside the library (SQUAD_NOALLOC_SCRATCH_BYTES).
+ *   - Limit: B*heads*n*d*sizeof(element) must fit in that array (bf16: at most
+ *     16,777,216 elements, fp32: 8,388,608); larger problems are rejected
+ *     with SQUAD_ERR_WORKSPACE before anything is launched.
+ *   - Every GPU that loads the library holds the array until the process
+ *     exits. The first call on a device looks up the array's device address
+ *     (a cudaGetSymbolAddress with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents. Each call overwrites every element it later reads, so nothing
+ *     needs clearing, but calls whose kernels overlap on the GPU (different
+ *     streams, or different host threads) race on the array: serialise them.
+ *   - Arguments and results are those of squad_attn_fwd with o1 == NULL;
+ *     lse1 and lse2 may be NULL. */
+#define SQUAD_NOALLOC_SCRATCH_BYTES (32u << 20)
+squad_status squad_attn_fwd_noalloc(const squad_desc* desc, const void* q, const void* k, const void* v,
+                                    void* o, float* lse1, float* lse2, void* stream);
+
 /* Backward of the forward for the loss sum(o * dout): writes dq, dk, dv.
  * o, o1, lse1, lse2 are the forward's outputs for the same q, k, v (all
  * required). The global pass is differentiated first (values o1), then the

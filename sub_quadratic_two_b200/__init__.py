@@ -227,3 +227,30 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tuple[int
               tile: Tuple[int, int, int], scale: Optional[float] = None) -> torch.Tensor:
     """SQuad-Attention of [B, heads, T*H*W, d] CUDA tensors (float32 or bfloat16), differentiable."""
     return _SquadAttention.apply(q, k, v, tuple(grid), tuple(tile), scale)
+
+
+def squad_attn_fwd_noalloc(q, k, v, grid, tile, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                           lse1: Optional[torch.Tensor] = None, lse2: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None):
+    """Forward for callers that cannot give the library scratch memory.
+
+    The C entry point squad_attn_fwd_noalloc allocates nothing: the local-pass
+    output lives in a fixed 32 MiB device array inside libsquad, so only inputs
+    and outputs are passed (here ``out`` is created with torch when not given).
+    Problems whose local-pass output does not fit are rejected with
+    SQUAD_ERR_WORKSPACE. Calls on one device share that array: do not let two of
+    them run on the GPU at the same time (different streams or threads).
+    """
+    lib = load_library()
+    fn = lib.squad_attn_fwd_noalloc
+    fn.argtypes = [ctypes.POINTER(SquadDesc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check_inputs(q, k, v)
+    desc = make_desc(q, grid, tile, scale)
+    o = torch.empty_like(q) if out is None else out
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse1), _ptr(lse2), st),
+               "squad_attn_fwd_noalloc")
+    return o

@@ -432,6 +432,65 @@ squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* 
   return simt_fwd<float>(g, q, k, val, out, lse, desc->d, p.scale, st);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- forward without allocation
+// Scratch for squad_attn_fwd_noalloc: the local-pass output of problems that fit.
+// Device code could name it directly, but the kernels take plain pointers, so the
+// host looks up its device address once per device (see noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_squad_noalloc_scratch[SQUAD_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a host-side stand-in, so the address must come from
+// cudaGetSymbolAddress, called with the device current; it is cached per device.
+squad_status noalloc_scratch(void** out) {
+  int dev = 0;
+  SQ_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return SQUAD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    SQ_CUDA(cudaGetSymbolAddress(&p, g_squad_noalloc_scratch));
+    if (p == nullptr) return cuda_fail(int(cudaErrorInvalidSymbol));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SQUAD_OK;
+}
+}  // namespace
+
+extern "C" squad_status squad_attn_fwd_noalloc(const squad_desc* desc, const void* q, const void* k, const void* v,
+                                               void* o, float* lse1, float* lse2, void* stream) {
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SQUAD_ERR_INVALID_ARG;
+  const size_t need = size_t(p.rows) * size_t(desc->d) * p.elem;
+  if (need > size_t(SQUAD_NOALLOC_SCRATCH_BYTES)) return SQUAD_ERR_WORKSPACE;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(lse1),
+                          static_cast<const void*>(lse2)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != SQUAD_OK) return s;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int d = desc->d;
+  // The local pass writes every element of the scratch that the global pass reads.
+  if (desc->dtype == SQUAD_BF16) {
+    if ((s = launch_fwd_tc(ds, d, p.g1, q, k, v, scratch, lse1, p.rows, p.scale, st)) != SQUAD_OK) return s;
+    return launch_fwd_tc(ds, d, p.g2, q, k, scratch, o, lse2, p.rows, p.scale, st);
+  }
+  if ((s = simt_fwd<float>(p.g1, q, k, v, scratch, lse1, d, p.scale, st)) != SQUAD_OK) return s;
+  return simt_fwd<float>(p.g2, q, k, scratch, o, lse2, d, p.scale, st);
+}
+
+extern "C" {
+
 squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k, const void* v, const void* o,
                             const void* o1, const float* lse1, const float* lse2, const void* dout, void* dq,
                             void* dk, void* dv, void* workspace, size_t workspace_bytes, void* stream) {

@@ -49,7 +49,8 @@ def parse_args():
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training-step leg")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget for the CPU baseline")
     ap.add_argument("--profile", action="store_true",
-                    help="profiling driver: one warm-up forward, then one forward (two kernel launches), no timing")
+                    help="profiling driver: one warm-up then one measured launch each of the fused forward, the "
+                         "local pass alone and the global pass alone; no timing")
     return ap.parse_args()
 
 
@@ -263,9 +264,12 @@ def main():
         sq.squad_attn_fwd(q, k, v, wl.grid, wl.tile, save=False, out=o, workspace=ws)
 
     if args.profile:
-        step()
-        torch.cuda.synchronize()
-        step()
+        o1p = torch.empty_like(q)
+        for _ in range(2):  # launch order: fused, local pass, global pass (twice)
+            step()
+            sq.squad_attn_fwd_pass(1, q, k, v, o1p, wl.grid, wl.tile)
+            sq.squad_attn_fwd_pass(2, q, k, o1p, o, wl.grid, wl.tile)
+            torch.cuda.synchronize()
         sq.poll_device_error()
         print("profile run done")
         return 0

@@ -67,14 +67,22 @@ typedef struct {
  * them). */
 
 /* Bytes of device workspace the call needs.
- *   which = 0: squad_attn_fwd with o1 == NULL (the local-pass output is kept
- *              there); with o1 != NULL the forward needs none.
+ *   which = 0: squad_attn_fwd with o1 == NULL: the local-pass output plus
+ *              B*heads progress counters (rounded up to 256 bytes each part).
+ *   which = 2: squad_attn_fwd with o1 != NULL: the counters only. With less
+ *              than this (e.g. no workspace) the forward still runs, as two
+ *              separate launches instead of one fused launch.
  *   which = 1: squad_attn_bwd (dO1 in the input dtype, the global-pass parts
  *              of dQ and dK in fp32, and two fp32 row vectors).
  * Returns SQUAD_OK and writes *bytes, or an argument/shape error. */
 squad_status squad_attn_workspace_size(const squad_desc* desc, int which, size_t* bytes);
 
 /* Forward: o = SQuad-Attention(q, k, v).
+ *   With enough workspace (see squad_attn_workspace_size) the bf16 path runs
+ *   as one launch in which the global pass of each (batch, head) starts as
+ *   soon as that head's local pass is done, while its Q, K and O1 are still in
+ *   L2; the counters in the workspace order the two. When o1 is NULL, the
+ *   local-pass rows are also dropped from L2 after their single use.
  *   o1   : [B,heads,n,d] local-pass output, written when non-NULL (needed by
  *          the backward); when NULL the workspace holds it.
  *   lse1 : [B,heads,n] local-pass log-sum-exp, written when non-NULL.

@@ -146,7 +146,10 @@ def squad_attn_fwd(q, k, v, grid, tile, scale: Optional[float] = None, save: boo
         o1 = torch.empty_like(q)
         lse1 = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
         lse2 = torch.empty(q.shape[:3], device=q.device, dtype=torch.float32)
-        ws, ws_bytes = None, 0
+        ws_bytes = workspace_size(desc, 2)
+        ws = workspace if workspace is not None else torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+        if ws.numel() * ws.element_size() < ws_bytes:
+            raise ValueError("workspace too small")
     else:
         o1 = lse1 = lse2 = None
         ws_bytes = workspace_size(desc, 0)

@@ -24,7 +24,8 @@ using sq::Geom;
 
 constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr int kMaxDevices = 64;
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+constexpr int kFusedLag = 2;  // see decode_item  // 2 s per wait: far above any legitimate wait
 
 thread_local int t_last_cuda = 0;
 
@@ -47,7 +48,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
-  bool fwd_attr_set[2][3] = {};  // [D=64/128][KT]
+  bool fwd_attr_set[2] = {};     // [D=64/128]
   bool bwd_attr_set[2][2][2] = {};  // [D=64/128][mode][out_f32]
 };
 
@@ -123,7 +124,10 @@ squad_status make_plan(const squad_desc* d, Plan* p) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-size_t fwd_workspace(const Plan& p, const squad_desc* d) { return align256(p.rows * d->d * p.elem); }
+// Forward workspace: [local-pass output, only when the caller passes no o1][per-head counters].
+size_t fwd_o1_bytes(const Plan& p, const squad_desc* d) { return align256(p.rows * d->d * p.elem); }
+size_t fwd_counter_bytes(const squad_desc* d) { return align256(size_t(d->B) * d->heads * sizeof(uint32_t)); }
+size_t fwd_workspace(const Plan& p, const squad_desc* d) { return fwd_o1_bytes(p, d) + fwd_counter_bytes(d); }
 
 struct BwdWs {
   size_t do1, dq2, dk2, D2, D1, total;
@@ -161,41 +165,80 @@ squad_status encode_map(CUtensorMap* m, const void* base, const Geom& g, int d, 
 
 // ---------------------------------------------------------------- launches
 
-template <int D, int KT>
-squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                             const CUtensorMap& mo, const sq::FwdArgs& a, cudaStream_t st) {
-  using Lay = sq::FwdLayout<D, KT>;
-  auto kern = sq::squad_fwd_tc_kernel<D, KT>;
-  bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0][KT];
+sq::PassArgs pass_args(const Geom& g, void* out, float* lse) {
+  sq::PassArgs pa{};
+  pa.g = g;
+  pa.out = out;
+  pa.lse = lse;
+  pa.jobs_per_bh = g.probs * g.nt;
+  pa.pairs_per_bh = (pa.jobs_per_bh + 1) / 2;
+  return pa;
+}
+
+template <int D>
+squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap* m, const sq::FwdArgs& a, cudaStream_t st) {
+  using Lay = sq::FwdLayout<D>;
+  auto kern = sq::squad_fwd_tc_kernel<D>;
+  bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0];
   if (!attr) {
     SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
     attr = true;
   }
-  const int grid = a.total_probs < ds->sms ? a.total_probs : ds->sms;
-  kern<<<grid, sq::kFwdThreads, Lay::ALLOC, st>>>(mq, mk, mv, mo, a);
-  SQ_CUDA(cudaGetLastError());
+  const int grid = a.total_items < ds->sms ? a.total_items : ds->sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(sq::kFwdThreads);
+  cfg.dynamicSmemBytes = Lay::ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  // The fused launch has CTAs wait on other CTAs' progress: require co-residency.
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = a.mode == sq::FWD_FUSED ? 1 : 0;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  SQ_CUDA(cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a));
   return SQUAD_OK;
 }
 
-squad_status launch_fwd_tc(DeviceState* ds, int d, const Geom& g, const void* q, const void* k, const void* val,
-                           void* out, float* lse, long long rows, float scale, cudaStream_t st) {
-  CUtensorMap mq, mk, mv, mo;
+// Forward launch. mode FWD_LOCAL: out1 = local pass of (q, k, val1). FWD_GLOBAL: out2 =
+// global pass of (q, k, val2). FWD_FUSED: both, the global pass reading out1 (= val2).
+squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, const void* q, const void* k,
+                           const void* val1, void* out1, float* lse1, const void* val2, void* out2, float* lse2,
+                           uint32_t* counters, const void* discard, cudaStream_t st) {
+  CUtensorMap m[8];
   squad_status s;
-  if ((s = encode_map(&mq, q, g, d, rows)) != SQUAD_OK) return s;
-  if ((s = encode_map(&mk, k, g, d, rows)) != SQUAD_OK) return s;
-  if ((s = encode_map(&mv, val, g, d, rows)) != SQUAD_OK) return s;
-  if ((s = encode_map(&mo, out, g, d, rows)) != SQUAD_OK) return s;
+  const bool do1 = mode != sq::FWD_GLOBAL, do2 = mode != sq::FWD_LOCAL;
+  if (do1) {
+    if ((s = encode_map(&m[0], q, p.g1, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[1], k, p.g1, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[2], val1, p.g1, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[3], out1, p.g1, d, p.rows)) != SQUAD_OK) return s;
+  }
+  if (do2) {
+    if ((s = encode_map(&m[4], q, p.g2, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[5], k, p.g2, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[6], val2, p.g2, d, p.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[7], out2, p.g2, d, p.rows)) != SQUAD_OK) return s;
+  }
+  for (int i = 0; i < 4; ++i) {  // the pass that does not run gets copies of valid maps
+    if (!do1) m[i] = m[4 + i];
+    if (!do2) m[4 + i] = m[i];
+  }
   sq::FwdArgs a{};
-  a.g = g;
-  a.total_probs = g.bh * g.probs;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.lse = lse;
+  a.ps[0] = pass_args(p.g1, out1, lse1);
+  a.ps[1] = pass_args(p.g2, out2, lse2);
+  a.mode = mode;
+  a.bh = p.g1.bh;
+  a.lag = kFusedLag < a.bh ? kFusedLag : a.bh;
+  a.total_items = (do1 ? a.bh * a.ps[0].pairs_per_bh : 0) + (do2 ? a.bh * a.ps[1].pairs_per_bh : 0);
+  a.scale_log2 = p.scale * 1.4426950408889634f;
+  a.counters = counters;
+  a.discard_base = static_cast<const uint8_t*>(discard);
   a.err = ds->err;
   a.timeout_ns = kWaitTimeoutNs;
-  const bool kt2 = g.nt >= 2;
-  if (d == 128) return kt2 ? launch_fwd_tc_t<128, 2>(ds, mq, mk, mv, mo, a, st)
-                           : launch_fwd_tc_t<128, 1>(ds, mq, mk, mv, mo, a, st);
-  return kt2 ? launch_fwd_tc_t<64, 2>(ds, mq, mk, mv, mo, a, st) : launch_fwd_tc_t<64, 1>(ds, mq, mk, mv, mo, a, st);
+  if (mode == sq::FWD_FUSED) SQ_CUDA(cudaMemsetAsync(counters, 0, size_t(a.bh) * sizeof(uint32_t), st));
+  if (d == 128) return launch_fwd_tc_t<128>(ds, m, a, st);
+  return launch_fwd_tc_t<64>(ds, m, a, st);
 }
 
 dim3 simt_grid(const Geom& g) { return dim3(unsigned(g.bh * g.probs), unsigned(sq::ceil_div(g.L, sq::kSimtWarps))); }
@@ -381,6 +424,8 @@ squad_status squad_attn_workspace_size(const squad_desc* desc, int which, size_t
   if (s != SQUAD_OK) return s;
   if (which == 0) {
     *bytes = fwd_workspace(p, desc);
+  } else if (which == 2) {
+    *bytes = fwd_counter_bytes(desc);
   } else if (which == 1) {
     *bytes = bwd_workspace(p, desc).total;
   } else {
@@ -396,20 +441,35 @@ squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k
   if (s != SQUAD_OK) return s;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return SQUAD_ERR_INVALID_ARG;
   void* o1buf = o1;
+  uint32_t* counters = nullptr;
   if (o1buf == nullptr) {
     if (workspace == nullptr || workspace_bytes < fwd_workspace(p, desc)) return SQUAD_ERR_WORKSPACE;
     o1buf = workspace;
+    counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + fwd_o1_bytes(p, desc));
+  } else if (workspace != nullptr && workspace_bytes >= fwd_counter_bytes(desc)) {
+    counters = static_cast<uint32_t*>(workspace);
   }
   for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(o1buf),
-                          static_cast<const void*>(lse1), static_cast<const void*>(lse2)})
+                          static_cast<const void*>(lse1), static_cast<const void*>(lse2),
+                          static_cast<const void*>(counters)})
     if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
   DeviceState* ds = nullptr;
   if ((s = device_state(&ds)) != SQUAD_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int d = desc->d;
   if (desc->dtype == SQUAD_BF16) {
-    if ((s = launch_fwd_tc(ds, d, p.g1, q, k, v, o1buf, lse1, p.rows, p.scale, st)) != SQUAD_OK) return s;
-    return launch_fwd_tc(ds, d, p.g2, q, k, o1buf, o, lse2, p.rows, p.scale, st);
+    if (counters != nullptr) {
+      // one launch: the global pass of each head runs right behind its local pass; without
+      // a caller o1 the local-pass rows are dropped from L2 once the global pass has read them
+      const bool drop = o1 == nullptr && (reinterpret_cast<uintptr_t>(o1buf) & 127u) == 0;
+      return launch_fwd_tc(ds, d, sq::FWD_FUSED, p, q, k, v, o1buf, lse1, o1buf, o, lse2, counters,
+                           drop ? o1buf : nullptr, st);
+    }
+    if ((s = launch_fwd_tc(ds, d, sq::FWD_LOCAL, p, q, k, v, o1buf, lse1, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, st)) != SQUAD_OK)
+      return s;
+    return launch_fwd_tc(ds, d, sq::FWD_GLOBAL, p, q, k, nullptr, nullptr, nullptr, o1buf, o, lse2, nullptr,
+                         nullptr, st);
   }
   if ((s = simt_fwd<float>(p.g1, q, k, v, o1buf, lse1, d, p.scale, st)) != SQUAD_OK) return s;
   return simt_fwd<float>(p.g2, q, k, o1buf, o, lse2, d, p.scale, st);
@@ -428,7 +488,13 @@ squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* 
   if ((s = device_state(&ds)) != SQUAD_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const Geom& g = stage == 1 ? p.g1 : p.g2;
-  if (desc->dtype == SQUAD_BF16) return launch_fwd_tc(ds, desc->d, g, q, k, val, out, lse, p.rows, p.scale, st);
+  if (desc->dtype == SQUAD_BF16) {
+    if (stage == 1)
+      return launch_fwd_tc(ds, desc->d, sq::FWD_LOCAL, p, q, k, val, out, lse, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, st);
+    return launch_fwd_tc(ds, desc->d, sq::FWD_GLOBAL, p, q, k, nullptr, nullptr, nullptr, val, out, lse, nullptr,
+                         nullptr, st);
+  }
   return simt_fwd<float>(g, q, k, val, out, lse, desc->d, p.scale, st);
 }
 
@@ -482,8 +548,11 @@ extern "C" squad_status squad_attn_fwd_noalloc(const squad_desc* desc, const voi
   const int d = desc->d;
   // The local pass writes every element of the scratch that the global pass reads.
   if (desc->dtype == SQUAD_BF16) {
-    if ((s = launch_fwd_tc(ds, d, p.g1, q, k, v, scratch, lse1, p.rows, p.scale, st)) != SQUAD_OK) return s;
-    return launch_fwd_tc(ds, d, p.g2, q, k, scratch, o, lse2, p.rows, p.scale, st);
+    if ((s = launch_fwd_tc(ds, d, sq::FWD_LOCAL, p, q, k, v, scratch, lse1, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, st)) != SQUAD_OK)
+      return s;
+    return launch_fwd_tc(ds, d, sq::FWD_GLOBAL, p, q, k, nullptr, nullptr, nullptr, scratch, o, lse2, nullptr,
+                         nullptr, st);
   }
   if ((s = simt_fwd<float>(p.g1, q, k, v, scratch, lse1, d, p.scale, st)) != SQUAD_OK) return s;
   return simt_fwd<float>(p.g2, q, k, scratch, o, lse2, d, p.scale, st);

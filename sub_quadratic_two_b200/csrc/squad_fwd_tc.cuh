@@ -1,28 +1,37 @@
-// squad_fwd_tc.cuh - forward of one SQuad-Attention pass on the sm_100a tensor cores.
+// squad_fwd_tc.cuh - forward of SQuad-Attention on the sm_100a tensor cores.
 //
-// One kernel serves both passes of the operator ("SQuad: Sub-Quadratic Attention
-// Distillation for Efficient Video Generation", gist.science technical summary,
-// Methodology section 1): the local pass (problems = windows, values = V, output
-// O1) and the global pass (problems = same-position groups across windows,
-// values = O1, output O). Only the tensor maps and the Geom differ.
+// The operator ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video
+// Generation", gist.science technical summary, Methodology section 1) is a local
+// pass (softmax attention inside each window, values V, output O1) followed by a
+// global pass (softmax attention among the tokens that share an in-window
+// position, same Q and K, values O1, output O). One kernel runs either pass, or
+// both in one launch with the global pass of a head scheduled right behind the
+// local pass of that head, so that its Q, K and O1 are still in L2.
 //
-// Design (B200):
-//   * Persistent CTAs, one per SM, loop over problems.
-//   * Warp-specialised: warp 4 issues TMA loads, warp 5 issues tcgen05.mma from
-//     one thread, warps 0-3 (128 threads, thread = TMEM lane = query row) run
-//     the softmax and the epilogue.
-//   * Every operand tile is a 5-D TMA box (d-block, a, b, c, token) cut from the
-//     problem box, so the strided gather of the global pass needs no permute:
-//     the box's strides walk across windows. Rows outside the problem are
-//     zero-filled by TMA on load and clipped on store.
-//   * S = Q K^T accumulates in TMEM (fp32, up to 256 key columns = two key
-//     tiles per group). The softmax reads S with tcgen05.ld, writes P as bf16
-//     back into the same TMEM columns, and O += P V runs with A = P read from
-//     TMEM (no shared-memory round trip for P). Problems with more than two
-//     key tiles run an online softmax across groups, rescaling O in TMEM.
-//   * The epilogue normalises O, packs bf16 into a 128B-swizzled staging tile
-//     and stores it with one TMA store per 64-column block; LSE is written
-//     per row.
+// Work decomposition. A problem (a window or a group) is cut into TMA boxes of at
+// most 128 rows (geometry.h). A job is one query box of one problem; it runs
+// over all key boxes of its problem with an online softmax. Jobs are taken in
+// pairs (A, B): A runs on softmax warpgroup 0, B on warpgroup 1, so that the
+// tensor core works on one while the other computes its softmax. When A and B
+// belong to the same problem (the 220-token windows: two query boxes) they share
+// the key and value boxes.
+//
+// Roles (384 threads):
+//   warps 0-3  softmax warpgroup 0, warps 4-7 softmax warpgroup 1
+//              (thread = TMEM lane = query row of the box)
+//   warp 8     TMA producer: Q, K and V boxes (rings of 2 each) in the order the
+//              tensor core consumes them; a Q box is released after its job's last S
+//   warps 9,11 one thread each issues tcgen05.mma for one softmax warpgroup:
+//              S = Q K^T (both operands K-major) and O += P V (P read from TMEM,
+//              V MN-major)
+//   warp 10    idle
+// The softmax warpgroups write their output rows straight from registers; in the
+// fused launch they also publish per-head completion of the local pass and, for
+// inference, drop the consumed local-pass rows from L2.
+// TMEM (512 columns): warpgroup a owns S/P at columns [256a, 256a+128) and O at
+// [256a+128, 256a+256). P overwrites S in place as packed bf16.
+// Every wait is bounded by the global timer; on expiry the CTA raises an abort
+// flag, lets its copies and MMAs in flight land, frees TMEM and returns.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -31,362 +40,442 @@
 
 namespace sq {
 
-struct FwdArgs {
+enum { FWD_LOCAL = 1, FWD_GLOBAL = 2, FWD_FUSED = 3 };
+
+struct PassArgs {
   Geom g;
-  int total_probs;      // g.bh * g.probs
-  float scale_log2;     // softmax scale * log2(e)
-  float* lse;           // [bh*n] natural-log LSE, or nullptr
-  int* err;             // device error word
-  uint64_t timeout_ns;  // bound for every wait
+  void* out;          // [rows, D] bf16 output of this pass
+  float* lse;         // natural-log LSE of this pass, or nullptr
+  int jobs_per_bh;    // problems per (batch, head) x boxes per problem
+  int pairs_per_bh;   // ceil(jobs_per_bh / 2)
 };
 
-constexpr int kFwdThreads = 192;
-constexpr int kTileRowsBytes = 128 * 128;  // one 64-column block of a 128-row tile (bf16)
+struct FwdArgs {
+  PassArgs ps[2];                // [0] local pass, [1] global pass
+  int mode;                      // FWD_LOCAL, FWD_GLOBAL or FWD_FUSED
+  int bh;                        // batch * heads
+  int lag;                       // FWD_FUSED: heads between a head's local pass and its global pass
+  int total_items;               // pairs over all (batch, head) and passes run
+  float scale_log2;              // softmax scale * log2(e)
+  uint32_t* counters;            // FWD_FUSED: finished local-pass jobs per (batch, head)
+  const uint8_t* discard_base;   // FWD_FUSED inference: local-pass output to drop from L2, or nullptr
+  int* err;
+  uint64_t timeout_ns;
+};
 
-template <int D, int KT>
+constexpr int kFwdThreads = 384;
+constexpr uint32_t kBlk = 128 * 128;  // one 64-column block of a 128-row bf16 box
+
+template <int D>
 struct FwdLayout {
-  static constexpr int DH = D / 64;                  // 64-column blocks per row
-  static constexpr int TILE = 128 * D * 2;           // bytes of one 128-row tile
-  static constexpr int Q_OFF = 0;                    // two Q tiles (double buffer)
-  static constexpr int K_OFF = Q_OFF + 2 * TILE;     // KT key tiles: [dh][KT*128 rows][128 B]
-  static constexpr int V_OFF = K_OFF + KT * TILE;    // KT value tiles, same layout
-  static constexpr int O_OFF = V_OFF + KT * TILE;    // output staging tile
-  static constexpr int BAR_OFF = O_OFF + TILE;
-  static constexpr int NBAR = 14;  // 13 used
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int NQ = 3, NK = 2, NV = 2;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + NQ * TILE;
+  static constexpr int V_OFF = K_OFF + NK * TILE;
+  static constexpr int BAR_OFF = V_OFF + NV * TILE;
+  static constexpr int NBAR = 24;
   static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
-  static constexpr int ALLOC = BYTES + 1024;          // alignment slack
-  static constexpr int TMEM_S = 0;                    // S / P columns
-  static constexpr int TMEM_O = 128 * KT;             // O accumulator columns
-  static constexpr int TMEM_COLS = (128 * KT + D) <= 256 ? 256 : 512;
+  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr int TMEM_COLS = 512;
 };
 
-enum { B_QFULL0 = 0, B_QFULL1, B_QEMPTY0, B_QEMPTY1, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_OFULL,
-       B_DRAIN, B_EPI };
+// barrier indices
+enum { F_QF = 0, F_QE = 3, F_KF = 6, F_KE = 8, F_VF = 10, F_VE = 12, F_SF = 14, F_PF = 16, F_OF = 18, F_ST = 20,
+       F_DRAIN = 22 };  // three Q slots, two of the rest (ring slot or warpgroup)
 
-__device__ __forceinline__ void flag_error(int* err, int code) {
-  if (err != nullptr) atomicCAS(err, 0, code);
+struct Item {
+  int pass, bh, pair;
+};
+
+// Work items in launch order. Fused: the local pass of heads 0..lag-1, then for each
+// later head h its local pass followed by the global pass of head h-lag, then the
+// global passes of the last lag heads. The lag gives the local pass of a head time
+// to finish everywhere before its global pass needs it, while its Q, K and O1 are
+// still in L2.
+__device__ __forceinline__ Item decode_item(const FwdArgs& a, int i) {
+  const int n1 = a.ps[0].pairs_per_bh, n2 = a.ps[1].pairs_per_bh;
+  if (a.mode == FWD_LOCAL) return {0, i / n1, i % n1};
+  if (a.mode == FWD_GLOBAL) return {1, i / n2, i % n2};
+  const int lag = a.lag;
+  if (i < lag * n1) return {0, i / n1, i % n1};
+  const int j = i - lag * n1, blk = j / (n1 + n2), r = j - blk * (n1 + n2);
+  if (blk < a.bh - lag) return r < n1 ? Item{0, blk + lag, r} : Item{1, blk, r - n1};
+  const int t = j - (a.bh - lag) * (n1 + n2);
+  return {1, a.bh - lag + t / n2, t % n2};
 }
 
-template <int D, int KT>
+struct Job {
+  bool valid;
+  int qt;    // query box within the problem
+  int prob;  // problem index over all (batch, head)
+  int base;  // first token of the problem
+};
+
+__device__ __forceinline__ Job job_of(const FwdArgs& a, const Item& it, int which) {
+  const PassArgs& p = a.ps[it.pass];
+  const int j = 2 * it.pair + which;
+  Job jb;
+  jb.valid = j < p.jobs_per_bh;
+  const int pl = j / p.g.nt;
+  jb.qt = j - pl * p.g.nt;
+  jb.prob = it.bh * p.g.probs + pl;
+  jb.base = jb.valid ? problem_base(p.g, jb.prob) : 0;
+  return jb;
+}
+
+__device__ __forceinline__ bool wait_counter(const uint32_t* c, uint32_t target, volatile int* abort,
+                                             uint64_t timeout_ns) {
+  if (ld_acquire_gpu(c) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu(c) >= target) return true;
+    __nanosleep(64);
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-    squad_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                        const FwdArgs args) {
-  using Lay = FwdLayout<D, KT>;
-  constexpr int DH = Lay::DH;
+    squad_fwd_tc_kernel(const __grid_constant__ CUtensorMap m0, const __grid_constant__ CUtensorMap m1,
+                        const __grid_constant__ CUtensorMap m2, const __grid_constant__ CUtensorMap m3,
+                        const __grid_constant__ CUtensorMap m4, const __grid_constant__ CUtensorMap m5,
+                        const __grid_constant__ CUtensorMap m6, const __grid_constant__ CUtensorMap m7,
+                        const __grid_constant__ FwdArgs args) {
+  using Lay = FwdLayout<D>;
+  constexpr int DH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::BAR_OFF + Lay::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::BAR_OFF + Lay::NBAR * 8 + 4);
+  // tensor map of (pass, role), role: 0 Q, 1 K, 2 values (selected without a local array)
+  auto map_of = [&](int pass, int role) -> const CUtensorMap* {
+    const int i = pass * 4 + role;
+    return i == 0 ? &m0 : i == 1 ? &m1 : i == 2 ? &m2 : i == 3 ? &m3 : i == 4 ? &m4 : i == 5 ? &m5 : i == 6 ? &m6 : &m7;
+  };
 
-  const Geom& g = args.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nt = g.nt;
-  const int ng = ceil_div(nt, KT);
-  const bool kv_resident = (ng == 1);  // key/value tiles loaded once per problem
   const uint64_t to = args.timeout_ns;
 
-  // Zero every operand buffer once: rows past the TMA box are never written and
-  // must stay finite (value rows are multiplied by P = 0).
+  // Rows past a TMA box are never written and must stay finite (values are multiplied by P = 0).
   {
     uint4* z = reinterpret_cast<uint4*>(smem);
     for (int i = threadIdx.x; i < Lay::BAR_OFF / 16; i += kFwdThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
   if (threadIdx.x == 0) {
-    mbar_init(&bars[B_QFULL0], 1);
-    mbar_init(&bars[B_QFULL1], 1);
-    mbar_init(&bars[B_QEMPTY0], 1);
-    mbar_init(&bars[B_QEMPTY1], 1);
-    mbar_init(&bars[B_KFULL], 1);
-    mbar_init(&bars[B_KEMPTY], 1);
-    mbar_init(&bars[B_VFULL], 1);
-    mbar_init(&bars[B_VEMPTY], 1);
-    mbar_init(&bars[B_SFULL], 1);
-    mbar_init(&bars[B_PFULL], 128);
-    mbar_init(&bars[B_OFULL], 1);
-    mbar_init(&bars[B_DRAIN], 1);
-    mbar_init(&bars[B_EPI], 128);
+    for (int i = 0; i < 3; ++i) {
+      mbar_init(&bars[F_QF + i], 1);
+      mbar_init(&bars[F_QE + i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[F_KF + i], 1);
+      mbar_init(&bars[F_KE + i], 2);
+      mbar_init(&bars[F_VF + i], 1);
+      mbar_init(&bars[F_VE + i], 2);
+      mbar_init(&bars[F_SF + i], 1);
+      mbar_init(&bars[F_PF + i], 128);
+      mbar_init(&bars[F_OF + i], 1);
+      mbar_init(&bars[F_ST + i], 128);
+    }
+    mbar_init(&bars[F_DRAIN], 1);
+    mbar_init(&bars[F_DRAIN + 1], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(tmem_holder, Lay::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_o);
-  }
+  if (warp == 8 && lane == 0)
+    for (int i = 0; i < 8; ++i) prefetch_tmap(map_of(i >> 2, i & 3));
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t sbase = smem_u32(smem);
+  const bool fused = args.mode == FWD_FUSED;
+  // launch: 384 x 168 registers; after: 2 x 128 x 224 (softmax) + 128 x 56 (control)
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 8) {
+    // ================================================================ TMA producer
     if (lane == 0) {
-      uint32_t q_iter = 0, kv_iter = 0;
-      const uint32_t tile_tx = uint32_t(g.box_rows) * D * 2;
+      uint32_t qc = 0, kc = 0, vc = 0;
       bool ok = true;
-      for (int prob = blockIdx.x; ok && prob < args.total_probs; prob += gridDim.x) {
-        const int base = problem_base(g, prob);
-        for (int qt = 0; ok && qt < nt; ++qt) {
-          const int b = q_iter & 1;
-          ok = mbar_wait(&bars[B_QEMPTY0 + b], ((q_iter >> 1) & 1) ^ 1, abort_flag, to);
-          if (!ok) break;
-          int b0, c0;
-          tile_origin(g, qt, b0, c0);
-          mbar_arrive_expect_tx(&bars[B_QFULL0 + b], tile_tx);
-#pragma unroll
-          for (int dh = 0; dh < DH; ++dh)
-            tma_load_5d(smem + Lay::Q_OFF + b * Lay::TILE + dh * kTileRowsBytes, &tm_q, &bars[B_QFULL0 + b],
-                        dh * 64, 0, b0, c0, base);
-          ++q_iter;
-          if (kv_resident && qt > 0) continue;
-          for (int grp = 0; ok && grp < ng; ++grp) {
-            const int kt0 = grp * KT, nkt = min(KT, nt - kt0);
-            ok = mbar_wait(&bars[B_KEMPTY], (kv_iter & 1) ^ 1, abort_flag, to);
-            if (!ok) break;
-            mbar_arrive_expect_tx(&bars[B_KFULL], tile_tx * nkt);
-            for (int j = 0; j < nkt; ++j) {
-              tile_origin(g, kt0 + j, b0, c0);
-#pragma unroll
+      for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
+        const Item it = decode_item(args, i);
+        const Geom& g = args.ps[it.pass].g;
+        const CUtensorMap* mq = map_of(it.pass, 0);
+        const CUtensorMap* mk = map_of(it.pass, 1);
+        const CUtensorMap* mv = map_of(it.pass, 2);
+        const Job J[2] = {job_of(args, it, 0), job_of(args, it, 1)};
+        const bool shared = J[1].valid && J[1].prob == J[0].prob;
+        const uint32_t tx = uint32_t(g.box_rows) * D * 2;
+        bool dep_done = !(fused && it.pass == 1);
+        for (int k = 0; ok && k < g.nt; ++k) {
+          for (int x = 0; ok && x < 2; ++x) {
+            if (!J[x].valid) continue;
+            int b0, c0;
+            if (k == 0) {
+              const uint32_t s = qc % 3;
+              if (!(ok = mbar_wait(&bars[F_QE + s], ((qc / 3) & 1) ^ 1, abort_flag, to))) break;
+              tile_origin(g, J[x].qt, b0, c0);
+              mbar_arrive_expect_tx(&bars[F_QF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::K_OFF + dh * KT * kTileRowsBytes + j * kTileRowsBytes, &tm_k,
-                            &bars[B_KFULL], dh * 64, 0, b0, c0, base);
+                tma_load_5d(smem + Lay::Q_OFF + s * Lay::TILE + dh * kBlk, mq, &bars[F_QF + s], dh * 64, 0, b0, c0,
+                            J[x].base);
+              ++qc;
             }
-            ok = mbar_wait(&bars[B_VEMPTY], (kv_iter & 1) ^ 1, abort_flag, to);
-            if (!ok) break;
-            mbar_arrive_expect_tx(&bars[B_VFULL], tile_tx * nkt);
-            for (int j = 0; j < nkt; ++j) {
-              tile_origin(g, kt0 + j, b0, c0);
-#pragma unroll
+            if (x == 1 && shared) continue;
+            tile_origin(g, k, b0, c0);
+            {
+              const uint32_t s = kc % 2;
+              if (!(ok = mbar_wait(&bars[F_KE + s], ((kc / 2) & 1) ^ 1, abort_flag, to))) break;
+              mbar_arrive_expect_tx(&bars[F_KF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::V_OFF + dh * KT * kTileRowsBytes + j * kTileRowsBytes, &tm_v,
-                            &bars[B_VFULL], dh * 64, 0, b0, c0, base);
+                tma_load_5d(smem + Lay::K_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KF + s], dh * 64, 0, b0, c0,
+                            J[x].base);
+              ++kc;
             }
-            ++kv_iter;
+            if (!dep_done) {
+              // the global pass of a head reads O1 only once the local pass of that head is complete
+              const uint32_t target = uint32_t(args.ps[0].jobs_per_bh);
+              if (!(ok = wait_counter(args.counters + it.bh, target, abort_flag, to))) break;
+              fence_async_global();
+              dep_done = true;
+            }
+            {
+              const uint32_t s = vc % 2;
+              if (!(ok = mbar_wait(&bars[F_VE + s], ((vc / 2) & 1) ^ 1, abort_flag, to))) break;
+              mbar_arrive_expect_tx(&bars[F_VF + s], tx);
+              for (int dh = 0; dh < DH; ++dh)
+                tma_load_5d(smem + Lay::V_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_VF + s], dh * 64, 0, b0, c0,
+                            J[x].base);
+              ++vc;
+            }
           }
         }
       }
-      // Let every load issued land before the CTA can exit.
-      for (int b = 0; b < 2; ++b) {
-        const uint32_t uses = q_iter > uint32_t(b) ? (q_iter - b + 1) / 2 : 0;
-        if (uses) mbar_wait_drain(&bars[B_QFULL0 + b], (uses - 1) & 1, to);
+      // let every issued load land before the CTA may exit
+      for (uint32_t s = 0; s < 3; ++s) {
+        const uint32_t uses = qc > s ? (qc - s + 2) / 3 : 0;
+        if (uses) mbar_wait_drain(&bars[F_QF + s], (uses - 1) & 1, to);
       }
-      if (kv_iter) {
-        mbar_wait_drain(&bars[B_KFULL], (kv_iter - 1) & 1, to);
-        mbar_wait_drain(&bars[B_VFULL], (kv_iter - 1) & 1, to);
+      for (uint32_t s = 0; s < 2; ++s) {
+        uint32_t uses = kc > s ? (kc - s + 1) / 2 : 0;
+        if (uses) mbar_wait_drain(&bars[F_KF + s], (uses - 1) & 1, to);
+        uses = vc > s ? (vc - s + 1) / 2 : 0;
+        if (uses) mbar_wait_drain(&bars[F_VF + s], (uses - 1) & 1, to);
       }
     }
-  } else if (warp == 5) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 9 || warp == 11) {
     if (lane == 0) {
-      uint32_t q_iter = 0, kv_iter = 0, pv_count = 0, p_iter = 0;
-      const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t tS = tmem + Lay::TMEM_S, tO = tmem + Lay::TMEM_O;
-      bool ok = true;
-      for (int prob = blockIdx.x; ok && prob < args.total_probs; prob += gridDim.x) {
-        for (int qt = 0; ok && qt < nt; ++qt) {
-          const int b = q_iter & 1;
-          ok = mbar_wait(&bars[B_QFULL0 + b], (q_iter >> 1) & 1, abort_flag, to);
-          if (!ok) break;
-          const uint32_t qaddr = sbase + Lay::Q_OFF + b * Lay::TILE;
-          for (int grp = 0; grp < ng; ++grp) {
-            const int kt0 = grp * KT, nkt = min(KT, nt - kt0);
-            const bool fresh = !(kv_resident && qt > 0);
-            const bool last_use = !kv_resident || qt == nt - 1;
-            if (fresh) {
-              ok = mbar_wait(&bars[B_KFULL], kv_iter & 1, abort_flag, to);
-              if (!ok) break;
-            }
-            // the previous P.V must have finished reading P before S is overwritten
-            if (pv_count > 0) {
-              ok = mbar_wait(&bars[B_OFULL], (pv_count - 1) & 1, abort_flag, to);
-              if (!ok) break;
-            }
-            tc_fence_after();
-            const uint32_t id_s = idesc_bf16_f32(128, 128 * nkt, 0, 0);
-            const uint32_t kaddr = sbase + Lay::K_OFF;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t koff = (kk >> 2) * kTileRowsBytes + (kk & 3) * 32;
-              const uint64_t ad = sdesc_sw128(qaddr + koff, 16, 1024);
-              const uint64_t bd = sdesc_sw128(kaddr + (kk >> 2) * KT * kTileRowsBytes + (kk & 3) * 32, 16, 1024);
-              mma_ss(tS, ad, bd, id_s, kk > 0 ? 1u : 0u);
-            }
-            tc_commit(&bars[B_SFULL]);
-            if (grp == ng - 1) tc_commit(&bars[B_QEMPTY0 + b]);
-            if (last_use) tc_commit(&bars[B_KEMPTY]);
-            ok = mbar_wait(&bars[B_PFULL], p_iter & 1, abort_flag, to);
-            if (!ok) break;
-            ++p_iter;
-            if (fresh) {
-              ok = mbar_wait(&bars[B_VFULL], kv_iter & 1, abort_flag, to);
-              if (!ok) break;
-            }
-            tc_fence_after();
-            const uint32_t vaddr = sbase + Lay::V_OFF;
-            for (int j = 0; j < nkt; ++j) {
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t bd = sdesc_sw128(vaddr + (j * 128 + kk * 16) * 128, KT * kTileRowsBytes, 1024);
-                mma_ts(tO, tS + j * 64 + kk * 8, bd, id_o, (grp > 0 || j > 0 || kk > 0) ? 1u : 0u);
-              }
-            }
-            tc_commit(&bars[B_OFULL]);
-            ++pv_count;
-            if (last_use) tc_commit(&bars[B_VEMPTY]);
-            if (fresh) ++kv_iter;
-          }
-          ++q_iter;
-        }
-      }
-      // all issued tensor-core work must finish before TMEM is released
-      tc_commit(&bars[B_DRAIN]);
-      mbar_wait_drain(&bars[B_DRAIN], 0, to);
-    }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 0-3)
-    const int row = threadIdx.x;  // TMEM lane == query row of the tile
-    const uint32_t lane_sel = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_sel + Lay::TMEM_S, tO = tmem + lane_sel + Lay::TMEM_O;
-    const float c2 = args.scale_log2;
-    uint32_t s_iter = 0, o_iter = 0, epi_iter = 0;
+    // ================================================================ MMA issuers
+    // One thread per softmax warpgroup (warp 9 serves jobs A, warp 11 jobs B), so each
+    // warpgroup's products are issued as soon as its own operands are ready and the two
+    // warpgroups settle into alternation: one computes its softmax while the tensor core
+    // runs the other's products. Key/value boxes are released after both users (the
+    // "empty" barriers count two arrivals; a box used by one job arrives twice).
+    const int x = warp == 9 ? 0 : 1;
+    const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);
+    const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
+    uint32_t ebase = 0, qbase = 0, pc = 0, pvc = 0;
     bool ok = true;
-    // warp-uniform bounded wait: tcgen05.ld/st are warp-collective, so all lanes
-    // must take the same branch after a wait
+    for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
+      const Item it = decode_item(args, i);
+      const int nk = args.ps[it.pass].g.nt;
+      const Job J0 = job_of(args, it, 0), J1 = job_of(args, it, 1);
+      const bool shared = J1.valid && J1.prob == J0.prob;
+      const uint32_t nvalid = uint32_t(J0.valid) + uint32_t(J1.valid);
+      const uint32_t nentries = shared ? uint32_t(nk) : uint32_t(nk) * nvalid;
+      if (x == 1 && !J1.valid) {
+        ebase += nentries;
+        qbase += nvalid;
+        continue;
+      }
+      const uint32_t q = qbase + uint32_t(x);
+      for (int k = 0; ok && k < nk; ++k) {
+        const uint32_t e = ebase + (shared ? uint32_t(k) : uint32_t(k) * nvalid + uint32_t(x));
+        const uint32_t slot = e & 1, par = (e >> 1) & 1;
+        if (!(ok = mbar_wait(&bars[F_KF + slot], par, abort_flag, to))) break;
+        if (k == 0 && !(ok = mbar_wait(&bars[F_QF + q % 3], (q / 3) & 1, abort_flag, to))) break;
+        // the previous P.V of this warpgroup has read P before S is overwritten
+        if (pvc > 0 && !(ok = mbar_wait(&bars[F_OF + x], (pvc - 1) & 1, abort_flag, to))) break;
+        tc_fence_after();
+        const uint32_t qa = sbase + Lay::Q_OFF + (q % 3) * Lay::TILE;
+        const uint32_t ka = sbase + Lay::K_OFF + slot * Lay::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk >> 2) * kBlk + (kk & 3) * 32;
+          mma_ss(tmem + x * 256, sdesc_sw128(qa + koff, 16, 1024), sdesc_sw128(ka + koff, 16, 1024), id_s,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[F_SF + x]);
+        if (k == nk - 1) tc_commit(&bars[F_QE + q % 3]);  // the job's Q box is no longer needed
+        tc_commit(&bars[F_KE + slot]);
+        if (!shared) tc_commit(&bars[F_KE + slot]);
+        if (!(ok = mbar_wait(&bars[F_PF + x], pc & 1, abort_flag, to))) break;
+        ++pc;
+        if (!(ok = mbar_wait(&bars[F_VF + slot], par, abort_flag, to))) break;
+        tc_fence_after();
+        const uint32_t va = sbase + Lay::V_OFF + slot * Lay::TILE;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, sdesc_sw128(va + kk * 16 * 128, kBlk, 1024), id_o,
+                 (k > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&bars[F_OF + x]);
+        ++pvc;
+        tc_commit(&bars[F_VE + slot]);
+        if (!shared) tc_commit(&bars[F_VE + slot]);
+      }
+      ebase += nentries;
+      qbase += nvalid;
+    }
+    tc_commit(&bars[F_DRAIN + x]);
+    mbar_wait_drain(&bars[F_DRAIN + x], 0, to);
+    }
+  } else if (warp == 10) {
+    // idle
+  } else {
+    // ================================================================ softmax warpgroups
+    const int a = warp >> 2;  // warpgroup: job A (0) or job B (1) of each pair
+    const int row = threadIdx.x & 127;
+    const uint32_t tS = tmem + (uint32_t((warp & 3) * 32) << 16) + a * 256;
+    const uint32_t tO = tS + 128;
+    const float c2 = args.scale_log2;
+    uint32_t sc = 0, pvseen = 0, pub = 0;
+    bool ok = true;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
-    // bounded rendezvous of the 128 softmax threads (an mbarrier, so it can time out)
-    auto epi_sync = [&]() -> bool {
-      mbar_arrive(&bars[B_EPI]);
-      const bool r = wwait(&bars[B_EPI], epi_iter & 1);
-      ++epi_iter;
-      return r;
-    };
-    for (int prob = blockIdx.x; ok && prob < args.total_probs; prob += gridDim.x) {
-      const int base = problem_base(g, prob);
-      for (int qt = 0; ok && qt < nt; ++qt) {
-        float m_run = -INFINITY, l_run = 0.f;
-        for (int grp = 0; grp < ng; ++grp) {
-          const int kt0 = grp * KT, nkt = min(KT, nt - kt0);
-          int vk[KT];
+    for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
+      const Item it = decode_item(args, i);
+      const PassArgs& P = args.ps[it.pass];
+      const Geom& g = P.g;
+      const Job J = job_of(args, it, a);
+      if (!J.valid) continue;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int k = 0; k < g.nt; ++k) {
+        if (!(ok = wwait(&bars[F_SF + a], sc & 1))) break;
+        ++sc;
+        tc_fence_after();
+        uint32_t r[128];
+        tmem_ld128(tS, r);
+        // key columns past the problem (a suffix of the box) -> -inf; only the ragged 32-column chunk is tested
+        const int lim = tile_valid_rows(g, k);
 #pragma unroll
-          for (int j = 0; j < KT; ++j) vk[j] = (j < nkt) ? tile_valid_rows(g, kt0 + j) : 0;
-          ok = wwait(&bars[B_SFULL], s_iter & 1);
-          if (!ok) break;
-          ++s_iter;
-          tc_fence_after();
-          // pass 1: row maximum over valid key columns
-          float mx = -INFINITY;
-          for (int c = 0; c < nkt * 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tS + c * 32, r);
-            const int lim = vk[c >> 2] - (c & 3) * 32;
+        for (int j = 0; j < 4; ++j) {
+          if (lim < 32 * (j + 1)) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (e < lim) mx = fmaxf(mx, __uint_as_float(r[e]));
+              if (32 * j + e >= lim) r[32 * j + e] = 0xff800000u;
           }
-          const float m_new = fmaxf(m_run, mx);
-          const float alpha = ex2_approx((m_run - m_new) * c2);
-          const float neg = -m_new * c2;
-          // pass 2: P = 2^(S*c2 - m*c2) as bf16 into the S columns already read
-          float sum = 0.f;
-          for (int c = 0; c < nkt * 4; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tS + c * 32, r);
-            const int lim = vk[c >> 2] - (c & 3) * 32;
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const float p0 = (e < lim) ? ex2_approx(fmaf(__uint_as_float(r[e]), c2, neg)) : 0.f;
-              const float p1 = (e + 1 < lim) ? ex2_approx(fmaf(__uint_as_float(r[e + 1]), c2, neg)) : 0.f;
-              sum += p0 + p1;
-              pk[e >> 1] = pack_bf16x2(p0, p1);
-            }
-            tmem_st16(tS + c * 16, pk);
-          }
-          tmem_st_wait();
-          if (grp > 0) {
-            // rescale the running O (after the previous P.V has landed)
-            ok = wwait(&bars[B_OFULL], o_iter & 1);
-            if (!ok) break;
-            ++o_iter;
-            tc_fence_after();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tO + c * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                tmem_st32(tO + c * 32, r);
-              }
-              tmem_st_wait();
-            }
-          }
-          tc_fence_before();
-          mbar_arrive(&bars[B_PFULL]);
-          l_run = l_run * alpha + sum;
-          m_run = m_new;
         }
-        if (!ok) break;
-        // ---------------- epilogue: O / l -> bf16 -> staging -> TMA store
-        ok = wwait(&bars[B_OFULL], o_iter & 1);
-        if (!ok) break;
-        ++o_iter;
-        tc_fence_after();
-        if (row == 0) bulk_wait_read0();  // previous store has finished reading the staging tile
-        ok = epi_sync();
-        if (!ok) break;
+        // row maximum: 8 independent partial maxima of three-input max
+        float mp[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mp[j] = fmaxf(__uint_as_float(r[j]), __uint_as_float(r[j + 8]));
+#pragma unroll
+        for (int e = 16; e < 128; e += 16)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) mp[j] = fmax3(mp[j], __uint_as_float(r[e + j]), __uint_as_float(r[e + j + 8]));
+        const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        // exact running maximum: the largest P of a row is exactly 1 before its bf16
+        // rounding, which keeps the dominant term of peaked rows exact
+        const float m_use = fmaxf(m_run, mx);
+        const float alpha = ex2_approx((m_run - m_use) * c2);
+        const float neg = -m_use * c2;
+        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // two 64-column halves: P of a half is packed and stored at once
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(r[64 * hh + e]), c2, neg));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(r[64 * hh + e + 1]), c2, neg));
+            sp[(e >> 1) & 7] += p0 + p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + hh * 32, pk);
+        }
+        const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        // the previous P.V has completed: S of this step was issued after it
+        if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {  // two 64-column halves keep register pressure down
+            uint32_t o[64];
+            tmem_ld64(tO + h * 64, o);
+#pragma unroll
+            for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st64(tO + h * 64, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars[F_PF + a]);
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16, each thread writes its own output row (16-byte stores)
+      pvseen += g.nt;
+      if (!(ok = wwait(&bars[F_OF + a], (pvseen - 1) & 1))) break;
+      tc_fence_after();
+      const int nvq = tile_valid_rows(g, J.qt);
+      const bool live = row < nvq;
+      const size_t tok = live ? size_t(J.base + tile_row_offset(g, J.qt, row)) : 0;
+      {
         const float inv = 1.f / l_run;
-        const uint32_t obase = sbase + Lay::O_OFF;
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(P.out) + tok * D * 2);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
-          const uint32_t blk = obase + (c >> 1) * kTileRowsBytes + row * 128;
+        for (int h = 0; h < D / 64; ++h) {
+          uint32_t o[64];
+          tmem_ld64(tO + h * 64, o);
+          if (live) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const int chunk = (c & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-            const uint32_t addr = blk + ((chunk ^ (row & 7)) << 4);
-            st_shared_v4(addr,
-                         pack_bf16x2(__uint_as_float(r[q4 * 8 + 0]) * inv, __uint_as_float(r[q4 * 8 + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(r[q4 * 8 + 2]) * inv, __uint_as_float(r[q4 * 8 + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(r[q4 * 8 + 4]) * inv, __uint_as_float(r[q4 * 8 + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(r[q4 * 8 + 6]) * inv, __uint_as_float(r[q4 * 8 + 7]) * inv));
+            for (int c = 0; c < 8; ++c)
+              dst[h * 8 + c] =
+                  make_uint4(pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                             pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                             pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                             pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
           }
-        }
-        fence_async_smem();
-        ok = epi_sync();
-        if (!ok) break;
-        int b0, c0;
-        tile_origin(g, qt, b0, c0);
-        if (row == 0) {
-#pragma unroll
-          for (int dh = 0; dh < DH; ++dh)
-            tma_store_5d(&tm_o, smem + Lay::O_OFF + dh * kTileRowsBytes, dh * 64, 0, b0, c0, base);
-          bulk_commit();
-        }
-        if (args.lse != nullptr && row < tile_valid_rows(g, qt)) {
-          const float lse2 = m_run * c2 + log2f(l_run);
-          args.lse[base + tile_row_offset(g, qt, row)] = lse2 * 0.69314718055994530942f;
         }
       }
+      tc_fence_before();
+      if (fused && it.pass == 0) {
+        // publish: every row of this job is written before the head's counter moves
+        mbar_arrive(&bars[F_ST + a]);
+        if (row == 0) {
+          ok = mbar_wait(&bars[F_ST + a], pub & 1, abort_flag, to);
+          fence_acq_rel_gpu();
+          fence_async_global();
+          red_release_gpu_add(args.counters + it.bh, 1u);
+        }
+        ++pub;
+        if (!(ok = __all_sync(0xffffffffu, ok) != 0)) break;
+      }
+      if (live && args.discard_base != nullptr && it.pass == 1 && g.nt == 1) {
+        // this row of the local-pass output was read once, as a value of this group: drop it from L2
+        const uint8_t* l1row = args.discard_base + tok * D * 2;
+#pragma unroll
+        for (int l = 0; l < D * 2 / 128; ++l) discard_l2_line(l1row + l * 128);
+      }
+      if (P.lse != nullptr && live)
+        P.lse[tok] = (m_run * c2 + log2f(l_run)) * 0.69314718055994530942f;
     }
-    if (row == 0) bulk_wait0();
   }
 
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) flag_error(args.err, 1);
-  if (warp == 5) {
+  if (*abort_flag && threadIdx.x == 0 && args.err != nullptr) atomicCAS(args.err, 0, 1);
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::TMEM_COLS);
   }

@@ -98,7 +98,9 @@ def test_backward_argument_errors(lib):
 def test_workspace_sizes(lib):
     d = _desc()
     rows = 1 * 2 * 256
-    assert sq.workspace_size(d, 0) == rows * 128 * 2
+    # local-pass output + one progress counter per (batch, head), each part 256-byte aligned
+    assert sq.workspace_size(d, 0) == rows * 128 * 2 + 256
+    assert sq.workspace_size(d, 2) == 256
     # dO1 (bf16) + dQ2, dK2 (fp32) + two fp32 row vectors, each 256-byte aligned
     assert sq.workspace_size(d, 1) == rows * 128 * 2 + 2 * rows * 128 * 4 + 2 * rows * 4
     with pytest.raises(sq.SquadError):

@@ -19,15 +19,16 @@
 // Roles (384 threads):
 //   warps 0-3  softmax warpgroup 0, warps 4-7 softmax warpgroup 1
 //              (thread = TMEM lane = query row of the box)
-//   warp 8     TMA producer: Q, K and V boxes (rings of 2 each) in the order the
-//              tensor core consumes them; a Q box is released after its job's last S
+//   warp 8     TMA producer: Q boxes (two slots, a box is released after its job's
+//              last S) and key/value boxes (one ring of five slots, K and V of a key
+//              box in consecutive slots) in the order the tensor core consumes them
 //   warps 9,11 one thread each issues tcgen05.mma for one softmax warpgroup:
 //              S = Q K^T (both operands K-major) and O += P V (P read from TMEM,
 //              V MN-major)
-//   warp 10    idle
-// The softmax warpgroups write their output rows straight from registers; in the
-// fused launch they also publish per-head completion of the local pass and, for
-// inference, drop the consumed local-pass rows from L2.
+//   warp 10    fused launch: publishes per-head completion of the local pass
+// The softmax warpgroups write their output rows (through a per-warp transpose patch,
+// so that stores are whole 128-byte lines) and, for inference, drop the consumed
+// local-pass rows from L2.
 // TMEM (512 columns): warpgroup a owns S/P at columns [256a, 256a+128) and O at
 // [256a+128, 256a+256). P overwrites S in place as packed bf16.
 // Every wait is bounded by the global timer; on expiry the CTA raises an abort
@@ -69,20 +70,21 @@ constexpr uint32_t kBlk = 128 * 128;  // one 64-column block of a 128-row bf16 b
 template <int D>
 struct FwdLayout {
   static constexpr int TILE = 128 * D * 2;
-  static constexpr int NQ = 3, NK = 2, NV = 2;
+  static constexpr int NQ = 2;   // Q boxes (released after the job's last S)
+  static constexpr int NKV = 4;  // one ring for key and value boxes, in consumption order
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + NQ * TILE;
-  static constexpr int V_OFF = K_OFF + NK * TILE;
-  static constexpr int BAR_OFF = V_OFF + NV * TILE;
+  static constexpr int KV_OFF = Q_OFF + NQ * TILE;
+  static constexpr int XP_OFF = KV_OFF + NKV * TILE;   // per softmax warp: 32 rows x 128 B transpose patch
+  static constexpr int BAR_OFF = XP_OFF + 8 * 4096;
   static constexpr int NBAR = 24;
-  static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
+  static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;  // + tmem holder, abort flag, two counters
   static constexpr int ALLOC = BYTES + 1024;
   static constexpr int TMEM_COLS = 512;
 };
 
 // barrier indices
-enum { F_QF = 0, F_QE = 3, F_KF = 6, F_KE = 8, F_VF = 10, F_VE = 12, F_SF = 14, F_PF = 16, F_OF = 18, F_ST = 20,
-       F_DRAIN = 22 };  // three Q slots, two of the rest (ring slot or warpgroup)
+enum { F_QF = 0, F_QE = 2, F_KVF = 4, F_KVE = 8, F_SF = 12, F_PF = 14, F_OF = 16, F_ST = 18, F_DRAIN = 20 };
+// (two Q slots, four key/value slots, two of the rest: one per warpgroup)
 
 struct Item {
   int pass, bh, pair;
@@ -124,6 +126,23 @@ __device__ __forceinline__ Job job_of(const FwdArgs& a, const Item& it, int whic
   return jb;
 }
 
+__device__ __forceinline__ bool wait_count_shared(const uint32_t* c, uint32_t target, volatile int* abort,
+                                                  uint64_t timeout_ns) {
+  if (ld_acquire_cta_shared(c) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_cta_shared(c) >= target) return true;
+    __nanosleep(32);
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > timeout_ns) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ bool wait_counter(const uint32_t* c, uint32_t target, volatile int* abort,
                                              uint64_t timeout_ns) {
   if (ld_acquire_gpu(c) >= target) return true;
@@ -155,6 +174,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::BAR_OFF);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::BAR_OFF + Lay::NBAR * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::BAR_OFF + Lay::NBAR * 8 + 4);
+  // per warpgroup: threads that finished writing their rows of local-pass jobs (monotonic)
+  uint32_t* rows_done = reinterpret_cast<uint32_t*>(smem + Lay::BAR_OFF + Lay::NBAR * 8 + 8);
   // tensor map of (pass, role), role: 0 Q, 1 K, 2 values (selected without a local array)
   auto map_of = [&](int pass, int role) -> const CUtensorMap* {
     const int i = pass * 4 + role;
@@ -170,15 +191,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = threadIdx.x; i < Lay::BAR_OFF / 16; i += kFwdThreads) z[i] = make_uint4(0, 0, 0, 0);
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) {
-      mbar_init(&bars[F_QF + i], 1);
-      mbar_init(&bars[F_QE + i], 1);
+    for (int i = 0; i < Lay::NKV; ++i) {
+      mbar_init(&bars[F_KVF + i], 1);
+      mbar_init(&bars[F_KVE + i], 2);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[F_KF + i], 1);
-      mbar_init(&bars[F_KE + i], 2);
-      mbar_init(&bars[F_VF + i], 1);
-      mbar_init(&bars[F_VE + i], 2);
+      mbar_init(&bars[F_QF + i], 1);
+      mbar_init(&bars[F_QE + i], 1);
       mbar_init(&bars[F_SF + i], 1);
       mbar_init(&bars[F_PF + i], 128);
       mbar_init(&bars[F_OF + i], 1);
@@ -187,6 +206,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&bars[F_DRAIN], 1);
     mbar_init(&bars[F_DRAIN + 1], 1);
     *abort_flag = 0;
+    rows_done[0] = 0;
+    rows_done[1] = 0;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -207,7 +228,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 8) {
     // ================================================================ TMA producer
     if (lane == 0) {
-      uint32_t qc = 0, kc = 0, vc = 0;
+      uint32_t qc = 0, uc = 0;  // Q boxes and key/value ring entries issued
       bool ok = true;
       for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
         const Item it = decode_item(args, i);
@@ -224,8 +245,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (!J[x].valid) continue;
             int b0, c0;
             if (k == 0) {
-              const uint32_t s = qc % 3;
-              if (!(ok = mbar_wait(&bars[F_QE + s], ((qc / 3) & 1) ^ 1, abort_flag, to))) break;
+              const uint32_t s = qc % 2;
+              if (!(ok = mbar_wait(&bars[F_QE + s], ((qc / 2) & 1) ^ 1, abort_flag, to))) break;
               tile_origin(g, J[x].qt, b0, c0);
               mbar_arrive_expect_tx(&bars[F_QF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
@@ -236,13 +257,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (x == 1 && shared) continue;
             tile_origin(g, k, b0, c0);
             {
-              const uint32_t s = kc % 2;
-              if (!(ok = mbar_wait(&bars[F_KE + s], ((kc / 2) & 1) ^ 1, abort_flag, to))) break;
-              mbar_arrive_expect_tx(&bars[F_KF + s], tx);
+              const uint32_t s = uc % Lay::NKV;
+              if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
+              mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::K_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KF + s], dh * 64, 0, b0, c0,
+                tma_load_5d(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KVF + s], dh * 64, 0, b0, c0,
                             J[x].base);
-              ++kc;
+              ++uc;
             }
             if (!dep_done) {
               // the global pass of a head reads O1 only once the local pass of that head is complete
@@ -252,27 +273,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               dep_done = true;
             }
             {
-              const uint32_t s = vc % 2;
-              if (!(ok = mbar_wait(&bars[F_VE + s], ((vc / 2) & 1) ^ 1, abort_flag, to))) break;
-              mbar_arrive_expect_tx(&bars[F_VF + s], tx);
+              const uint32_t s = uc % Lay::NKV;
+              if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
+              mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::V_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_VF + s], dh * 64, 0, b0, c0,
+                tma_load_5d(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_KVF + s], dh * 64, 0, b0, c0,
                             J[x].base);
-              ++vc;
+              ++uc;
             }
           }
         }
       }
       // let every issued load land before the CTA may exit
-      for (uint32_t s = 0; s < 3; ++s) {
-        const uint32_t uses = qc > s ? (qc - s + 2) / 3 : 0;
+      for (uint32_t s = 0; s < 2; ++s) {
+        const uint32_t uses = qc > s ? (qc - s + 1) / 2 : 0;
         if (uses) mbar_wait_drain(&bars[F_QF + s], (uses - 1) & 1, to);
       }
-      for (uint32_t s = 0; s < 2; ++s) {
-        uint32_t uses = kc > s ? (kc - s + 1) / 2 : 0;
-        if (uses) mbar_wait_drain(&bars[F_KF + s], (uses - 1) & 1, to);
-        uses = vc > s ? (vc - s + 1) / 2 : 0;
-        if (uses) mbar_wait_drain(&bars[F_VF + s], (uses - 1) & 1, to);
+      for (uint32_t s = 0; s < uint32_t(Lay::NKV); ++s) {
+        const uint32_t uses = uc > s ? (uc - s + Lay::NKV - 1) / Lay::NKV : 0;
+        if (uses) mbar_wait_drain(&bars[F_KVF + s], (uses - 1) & 1, to);
       }
     }
   } else if (warp == 9 || warp == 11) {
@@ -302,15 +321,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       const uint32_t q = qbase + uint32_t(x);
       for (int k = 0; ok && k < nk; ++k) {
+        // key/value entry of this job's key box k; K and V of an entry are consecutive ring slots
         const uint32_t e = ebase + (shared ? uint32_t(k) : uint32_t(k) * nvalid + uint32_t(x));
-        const uint32_t slot = e & 1, par = (e >> 1) & 1;
-        if (!(ok = mbar_wait(&bars[F_KF + slot], par, abort_flag, to))) break;
-        if (k == 0 && !(ok = mbar_wait(&bars[F_QF + q % 3], (q / 3) & 1, abort_flag, to))) break;
+        const uint32_t uk = 2 * e, uv = 2 * e + 1;
+        const uint32_t ks = uk % Lay::NKV, vs = uv % Lay::NKV;
+        if (!(ok = mbar_wait(&bars[F_KVF + ks], (uk / Lay::NKV) & 1, abort_flag, to))) break;
+        if (k == 0 && !(ok = mbar_wait(&bars[F_QF + q % 2], (q / 2) & 1, abort_flag, to))) break;
         // the previous P.V of this warpgroup has read P before S is overwritten
         if (pvc > 0 && !(ok = mbar_wait(&bars[F_OF + x], (pvc - 1) & 1, abort_flag, to))) break;
         tc_fence_after();
-        const uint32_t qa = sbase + Lay::Q_OFF + (q % 3) * Lay::TILE;
-        const uint32_t ka = sbase + Lay::K_OFF + slot * Lay::TILE;
+        const uint32_t qa = sbase + Lay::Q_OFF + (q % 2) * Lay::TILE;
+        const uint32_t ka = sbase + Lay::KV_OFF + ks * Lay::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * kBlk + (kk & 3) * 32;
@@ -318,22 +339,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars[F_SF + x]);
-        if (k == nk - 1) tc_commit(&bars[F_QE + q % 3]);  // the job's Q box is no longer needed
-        tc_commit(&bars[F_KE + slot]);
-        if (!shared) tc_commit(&bars[F_KE + slot]);
+        if (k == nk - 1) tc_commit(&bars[F_QE + q % 2]);  // the job's Q box is no longer needed
+        tc_commit(&bars[F_KVE + ks]);
+        if (!shared) tc_commit(&bars[F_KVE + ks]);
         if (!(ok = mbar_wait(&bars[F_PF + x], pc & 1, abort_flag, to))) break;
         ++pc;
-        if (!(ok = mbar_wait(&bars[F_VF + slot], par, abort_flag, to))) break;
+        if (!(ok = mbar_wait(&bars[F_KVF + vs], (uv / Lay::NKV) & 1, abort_flag, to))) break;
         tc_fence_after();
-        const uint32_t va = sbase + Lay::V_OFF + slot * Lay::TILE;
+        const uint32_t va = sbase + Lay::KV_OFF + vs * Lay::TILE;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, sdesc_sw128(va + kk * 16 * 128, kBlk, 1024), id_o,
                  (k > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&bars[F_OF + x]);
         ++pvc;
-        tc_commit(&bars[F_VE + slot]);
-        if (!shared) tc_commit(&bars[F_VE + slot]);
+        tc_commit(&bars[F_KVE + vs]);
+        if (!shared) tc_commit(&bars[F_KVE + vs]);
       }
       ebase += nentries;
       qbase += nvalid;
@@ -342,7 +363,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_wait_drain(&bars[F_DRAIN + x], 0, to);
     }
   } else if (warp == 10) {
-    // idle
+    // ================================================================ publisher (fused launch)
+    // Once all rows of a local-pass job are written (the warpgroup's 128 threads each add
+    // one to rows_done after their stores), make them visible at GPU scope and count the job for its
+    // head; the global pass of that head starts when its count is complete. Done here so
+    // the softmax warpgroups never wait for the fence.
+    if (fused && lane == 0) {
+      uint32_t pub[2] = {0, 0};
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
+        const Item it = decode_item(args, i);
+        if (it.pass != 0) continue;
+        for (int x = 0; ok && x < 2; ++x) {
+          if (!job_of(args, it, x).valid) continue;
+          ++pub[x];
+          if (!(ok = wait_count_shared(&rows_done[x], 128u * pub[x], abort_flag, to))) break;
+          fence_acq_rel_gpu();
+          red_release_gpu_add(args.counters + it.bh, 1u);
+        }
+      }
+    }
   } else {
     // ================================================================ softmax warpgroups
     const int a = warp >> 2;  // warpgroup: job A (0) or job B (1) of each pair
@@ -350,7 +390,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const uint32_t tS = tmem + (uint32_t((warp & 3) * 32) << 16) + a * 256;
     const uint32_t tO = tS + 128;
     const float c2 = args.scale_log2;
-    uint32_t sc = 0, pvseen = 0, pub = 0;
+    uint32_t sc = 0, pvseen = 0;
     bool ok = true;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
@@ -432,36 +472,37 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool live = row < nvq;
       const size_t tok = live ? size_t(J.base + tile_row_offset(g, J.qt, row)) : 0;
       {
+        // Each thread holds its own row. A warp passes its 32 rows through a private
+        // 128B-swizzled patch so that every global store writes four whole 128-byte lines.
         const float inv = 1.f / l_run;
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(P.out) + tok * D * 2);
-#pragma unroll
+        const uint32_t xp = sbase + Lay::XP_OFF + (warp & 7) * 4096;
+        const int lr = lane >> 3, lc = lane & 7;  // read-back: row 4*i + lr, 16-byte chunk lc
+        uint8_t* outb = static_cast<uint8_t*>(P.out);
+#pragma unroll 1
         for (int h = 0; h < D / 64; ++h) {
           uint32_t o[64];
           tmem_ld64(tO + h * 64, o);
-          if (live) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              dst[h * 8 + c] =
-                  make_uint4(pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
-                             pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
-                             pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
-                             pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
+                         pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
+                         pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
+                         pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + lr;  // row of this warp (lane r owns it)
+            const size_t rtok = __shfl_sync(0xffffffffu, tok, r);
+            const bool rlive = __shfl_sync(0xffffffffu, live, r);
+            const uint4 val = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
+            if (rlive) *reinterpret_cast<uint4*>(outb + rtok * D * 2 + h * 128 + lc * 16) = val;
           }
+          __syncwarp();
         }
       }
       tc_fence_before();
-      if (fused && it.pass == 0) {
-        // publish: every row of this job is written before the head's counter moves
-        mbar_arrive(&bars[F_ST + a]);
-        if (row == 0) {
-          ok = mbar_wait(&bars[F_ST + a], pub & 1, abort_flag, to);
-          fence_acq_rel_gpu();
-          fence_async_global();
-          red_release_gpu_add(args.counters + it.bh, 1u);
-        }
-        ++pub;
-        if (!(ok = __all_sync(0xffffffffu, ok) != 0)) break;
-      }
+      if (fused && it.pass == 0) red_release_cta_shared_add(&rows_done[a], 1u);  // warp 10 publishes
       if (live && args.discard_base != nullptr && it.pass == 1 && g.nt == 1) {
         // this row of the local-pass output was read once, as a value of this group: drop it from L2
         const uint8_t* l1row = args.discard_base + tok * D * 2;

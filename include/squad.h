@@ -144,6 +144,14 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
  * online-softmax group. No CUDA call is made. */
 squad_status squad_plan_info(const squad_desc* desc, int stage, int* info);
 
+/* Self-test of the device timeout path (no counterpart in the paper): launches
+ * one small kernel whose thread waits, through the same bounded wait the
+ * attention kernels use, on a barrier that nothing ever completes. After
+ * timeout_ns (1 us .. 10 s) it gives up and sets the device error word, so a
+ * following squad_poll_device_error returns SQUAD_ERR_TIMEOUT and clears it.
+ * Nothing faults or hangs and the context stays usable. */
+squad_status squad_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word. Returns SQUAD_ERR_TIMEOUT if a kernel gave up on a bounded wait since
  * the last poll, SQUAD_ERR_CUDA if the synchronisation failed, else SQUAD_OK. */

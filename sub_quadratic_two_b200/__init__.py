@@ -201,6 +201,15 @@ def squad_attn_bwd(q, k, v, o, o1, lse1, lse2, dout, grid, tile, scale: Optional
     return dq, dk, dv
 
 
+def selftest_wait_timeout(timeout_ns: int = 10_000_000, stream: Optional[torch.cuda.Stream] = None):
+    """Launch the device timeout self-test (a bounded wait that nothing satisfies)."""
+    lib = load_library()
+    lib.squad_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, ctypes.c_void_p]
+    lib.squad_selftest_wait_timeout.restype = ctypes.c_int
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib.squad_selftest_wait_timeout(int(timeout_ns), _stream_handle(stream, dev)), "squad_selftest_wait_timeout")
+
+
 def poll_device_error(stream: Optional[torch.cuda.Stream] = None, device=None):
     """Synchronise and raise SquadError(SQUAD_ERR_TIMEOUT) if a kernel gave up on a wait."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)

@@ -413,6 +413,20 @@ squad_status simt_bwd(const Plan& p, const BwdWs& w, uint8_t* ws, const void* q,
 
 }  // namespace
 
+// One thread waits on a barrier that nothing completes: the bounded wait gives up
+// after timeout_ns and the error word is set (the test of the device timeout path).
+__global__ void selftest_timeout_kernel(int* err, uint64_t timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sq::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sq::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !sq::mbar_wait(&bar, 0, &abort_flag, timeout_ns)) atomicCAS(err, 0, 1);
+}
+
 // ==================================================================== C ABI
 
 extern "C" {
@@ -599,6 +613,16 @@ squad_status squad_plan_info(const squad_desc* desc, int stage, int* info) {
   info[5] = g.b_sub;
   info[6] = g.c_sub;
   info[7] = g.nt >= 2 ? 2 : 1;
+  return SQUAD_OK;
+}
+
+squad_status squad_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return SQUAD_ERR_INVALID_ARG;
+  DeviceState* ds = nullptr;
+  squad_status s;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(ds->err, timeout_ns);
+  SQ_CUDA(cudaGetLastError());
   return SQUAD_OK;
 }
 

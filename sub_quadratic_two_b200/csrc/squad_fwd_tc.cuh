@@ -90,6 +90,7 @@ struct Item {
   int pass, bh, pair;
 };
 
+
 // Work items in launch order. Fused: the local pass of heads 0..lag-1, then for each
 // later head h its local pass followed by the global pass of head h-lag, then the
 // global passes of the last lag heads. The lag gives the local pass of a head time
@@ -229,6 +230,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ================================================================ TMA producer
     if (lane == 0) {
       uint32_t qc = 0, uc = 0;  // Q boxes and key/value ring entries issued
+      // L2 policies in the fused launch: the local pass's Q and K are read again by the
+      // global pass (keep), its V is not (drop first); the global pass is their last use.
+      const uint64_t pol_keep = make_policy_evict_last(), pol_drop = make_policy_evict_first();
+      const uint64_t pol_norm = make_policy_evict_normal();
       bool ok = true;
       for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
         const Item it = decode_item(args, i);
@@ -240,6 +245,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const bool shared = J[1].valid && J[1].prob == J[0].prob;
         const uint32_t tx = uint32_t(g.box_rows) * D * 2;
         bool dep_done = !(fused && it.pass == 1);
+        const uint64_t pol_qk = !fused ? pol_norm : it.pass == 0 ? pol_keep : pol_drop;
+        const uint64_t pol_v = !fused ? pol_norm : pol_drop;
         for (int k = 0; ok && k < g.nt; ++k) {
           for (int x = 0; ok && x < 2; ++x) {
             if (!J[x].valid) continue;
@@ -250,8 +257,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tile_origin(g, J[x].qt, b0, c0);
               mbar_arrive_expect_tx(&bars[F_QF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::Q_OFF + s * Lay::TILE + dh * kBlk, mq, &bars[F_QF + s], dh * 64, 0, b0, c0,
-                            J[x].base);
+                tma_load_5d_hint(smem + Lay::Q_OFF + s * Lay::TILE + dh * kBlk, mq, &bars[F_QF + s], dh * 64, 0, b0,
+                                 c0, J[x].base, pol_qk);
               ++qc;
             }
             if (x == 1 && shared) continue;
@@ -261,8 +268,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
               mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KVF + s], dh * 64, 0, b0, c0,
-                            J[x].base);
+                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KVF + s], dh * 64, 0, b0,
+                                 c0, J[x].base, pol_qk);
               ++uc;
             }
             if (!dep_done) {
@@ -277,8 +284,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
               mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_KVF + s], dh * 64, 0, b0, c0,
-                            J[x].base);
+                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_KVF + s], dh * 64, 0, b0,
+                                 c0, J[x].base, pol_v);
               ++uc;
             }
           }
@@ -477,6 +484,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float inv = 1.f / l_run;
         const uint32_t xp = sbase + Lay::XP_OFF + (warp & 7) * 4096;
         const int lr = lane >> 3, lc = lane & 7;  // read-back: row 4*i + lr, 16-byte chunk lc
+        // fused launch: O1 rows are read again by the global pass (keep); O rows are final (drop first)
+        const uint64_t pol_out = !fused ? make_policy_evict_normal()
+                                 : it.pass == 0 ? make_policy_evict_last() : make_policy_evict_first();
         uint8_t* outb = static_cast<uint8_t*>(P.out);
 #pragma unroll 1
         for (int h = 0; h < D / 64; ++h) {
@@ -496,7 +506,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const size_t rtok = __shfl_sync(0xffffffffu, tok, r);
             const bool rlive = __shfl_sync(0xffffffffu, live, r);
             const uint4 val = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
-            if (rlive) *reinterpret_cast<uint4*>(outb + rtok * D * 2 + h * 128 + lc * 16) = val;
+            if (rlive) st_global_v4_hint(outb + rtok * D * 2 + h * 128 + lc * 16, val, pol_out);
           }
           __syncwarp();
         }

@@ -136,6 +136,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ helpers
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """TFLOP/s of the whole job when every rank runs one workload per step (weak scaling)."""
+    return world * flops_per_rank_step / (ms_per_step / 1e3) / 1e12
+
+
 def source_sha(path: str) -> str:
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
@@ -245,13 +261,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     if args.profile_bwd:
         twl = WORKLOADS["wan5b_train"]
         tin = make_inputs(twl)
@@ -312,9 +321,9 @@ def main():
     sampler.stop()
     sq.poll_device_error()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = max_over_ranks(sum(step_ms))
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops / (ms_per_step / 1e3) / 1e12
+    value = whole_job_throughput(world, flops, ms_per_step)
     clocks = sampler.summary(t_wall0, t_wall1)
 
     # ---------------- per-pass kernel timing (same stream, events, L2 flushed)
@@ -381,8 +390,8 @@ def main():
             b.record(stream)
             torch.cuda.synchronize()
             barrier()
-        e2e_ms = max_over_ranks(a.elapsed_time(b)) / ek
-        e2e = {"value": world * flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+        e2e_ms = max_over_ranks(a.elapsed_time(b), dev) / ek
+        e2e = {"value": whole_job_throughput(world, flops, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * hq.numel() * hq.element_size(),
                "d2h_bytes_per_step": ho.numel() * ho.element_size(), "steps": ek,
                "path": "sub_quadratic_two_b200.attention on pinned host tensors"}
@@ -412,9 +421,9 @@ def main():
         torch.cuda.synchronize()
         barrier()
         sq.poll_device_error()
-        tms = max_over_ranks(a.elapsed_time(b)) / tsteps
+        tms = max_over_ranks(a.elapsed_time(b), dev) / tsteps
         tfl = twl.fwd_flops() + twl.bwd_flops()
-        train = {"workload": twl.name, "ms_per_step": tms, "TFLOP/s": world * tfl / (tms / 1e3) / 1e12,
+        train = {"workload": twl.name, "ms_per_step": tms, "TFLOP/s": whole_job_throughput(world, tfl, tms),
                  "useful_flops_per_step": tfl, "steps": tsteps,
                  "note": "backward: tcgen05 dq and dk/dv kernels per pass"}
         del tq, tk, tv, tdo

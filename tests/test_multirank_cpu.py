@@ -1,0 +1,70 @@
+"""The multi-rank path of bench.py on CPU (gloo, world size 2).
+
+With N GPUs every rank runs the whole workload on its own GPU (independent
+(batch, head) problems, weak scaling); the only cross-rank communication is
+the barrier and the max over ranks of the timings. Both are host logic and run
+here on gloo.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dist.barrier()
+        slowest = bench.max_over_ranks(1.0 + 2.5 * rank)          # per-rank step times (ms)
+        tput = bench.whole_job_throughput(world, 1.0e11, slowest)
+        out.put((rank, slowest, tput))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_throughput_gloo():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, slowest, tput in res:
+        assert slowest == pytest.approx(3.5)                      # every rank sees the slowest rank
+        assert tput == pytest.approx(2 * 1.0e11 / 3.5e-3 / 1e12)  # whole-job TFLOP/s over both ranks
+
+
+def test_single_process_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(4.2) == 4.2
+    assert bench.whole_job_throughput(1, 1.0e12, 1000.0) == pytest.approx(1.0)
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""

@@ -14,6 +14,7 @@
 
 #include "squad.h"
 #include "geometry.h"
+#include "squad_bwd_fused.cuh"
 #include "squad_bwd_tc.cuh"
 #include "squad_fwd_tc.cuh"
 #include "squad_simt.cuh"
@@ -50,6 +51,7 @@ struct DeviceState {
   int* err = nullptr;          // device address of g_squad_dev_err
   bool fwd_attr_set[2] = {};     // [D=64/128]
   bool bwd_attr_set[2][2][2] = {};  // [D=64/128][mode][out_f32]
+  bool fused_attr_set[2][2] = {};   // [D=64/128][out_f32]
 };
 
 std::mutex g_mu;
@@ -326,6 +328,22 @@ squad_status launch_bwd_tc_t(DeviceState* ds, const CUtensorMap* maps, const sq:
   return SQUAD_OK;
 }
 
+template <int D, bool F32>
+squad_status launch_bwd_fused_t(DeviceState* ds, const CUtensorMap* maps, const sq::BwdFusedArgs& a,
+                                cudaStream_t st) {
+  using Lay = sq::BwdFusedLayout<D>;
+  auto kern = sq::squad_bwd_fused_kernel<D, F32>;
+  bool& attr = ds->fused_attr_set[D == 128 ? 1 : 0][F32 ? 1 : 0];
+  if (!attr) {
+    SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
+    attr = true;
+  }
+  const int grid = a.total_items < ds->sms ? a.total_items : ds->sms;
+  kern<<<grid, sq::kBwdFusedThreads, Lay::ALLOC, st>>>(maps[0], maps[1], maps[2], maps[3], a);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
 template <int MODE, bool F32>
 squad_status launch_bwd_tc(DeviceState* ds, int d, const CUtensorMap* maps, const sq::BwdArgs& a, cudaStream_t st) {
   if (d == 128) return launch_bwd_tc_t<128, MODE, F32>(ds, maps, a, st);
@@ -353,6 +371,26 @@ squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, c
   if ((s = encode_map(&maps[1], k, g, d, p.rows)) != SQUAD_OK) return s;
   if ((s = encode_map(&maps[2], val, g, d, p.rows)) != SQUAD_OK) return s;
   if ((s = encode_map(&maps[3], dout, g, d, p.rows)) != SQUAD_OK) return s;
+  if (g.nt == 1) {
+    // every problem is one box: one kernel computes dq, dk and dval from one S and one dP
+    sq::BwdFusedArgs f{};
+    f.g = g;
+    f.total_items = g.bh * g.probs;
+    f.scale = p.scale;
+    f.scale_log2 = p.scale * 1.4426950408889634f;
+    f.lse = lse;
+    f.Drow = Drow;
+    f.add_q = dq_add;
+    f.add_k = dk_add;
+    f.out_q = dq;
+    f.out_k = dk;
+    f.out_val = dval;
+    f.err = ds->err;
+    f.timeout_ns = kWaitTimeoutNs;
+    if (d == 128)
+      return f32_out ? launch_bwd_fused_t<128, true>(ds, maps, f, st) : launch_bwd_fused_t<128, false>(ds, maps, f, st);
+    return f32_out ? launch_bwd_fused_t<64, true>(ds, maps, f, st) : launch_bwd_fused_t<64, false>(ds, maps, f, st);
+  }
   sq::BwdArgs a{};
   a.g = g;
   a.total_items = g.bh * g.probs * g.nt;

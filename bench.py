@@ -425,7 +425,7 @@ def main():
         tfl = twl.fwd_flops() + twl.bwd_flops()
         train = {"workload": twl.name, "ms_per_step": tms, "TFLOP/s": whole_job_throughput(world, tfl, tms),
                  "useful_flops_per_step": tfl, "steps": tsteps,
-                 "note": "backward: one fused tcgen05 kernel for a pass whose problems fit one 128-row box (global pass), tcgen05 dq and dk/dv kernels otherwise (local pass)"}
+                 "note": "backward: one fused tcgen05 kernel per pass (dQ parts of multi-box problems added with vector reductions, then one fp32-to-bf16 pass)"}
         del tq, tk, tv, tdo
 
     # ---------------- CPU baseline: the oracle on host cores, rank 0 at N=1 only

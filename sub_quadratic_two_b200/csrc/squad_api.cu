@@ -15,7 +15,6 @@
 #include "squad.h"
 #include "geometry.h"
 #include "squad_bwd_fused.cuh"
-#include "squad_bwd_tc.cuh"
 #include "squad_fwd_tc.cuh"
 #include "squad_simt.cuh"
 
@@ -50,7 +49,6 @@ struct DeviceState {
   int sms = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
   bool fwd_attr_set[2] = {};     // [D=64/128]
-  bool bwd_attr_set[2][2][2] = {};  // [D=64/128][mode][out_f32]
   bool fused_attr_set[2][2] = {};   // [D=64/128][out_f32]
 };
 
@@ -66,6 +64,9 @@ squad_status device_state(DeviceState** out) {
   int dev = 0;
   SQ_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return SQUAD_ERR_UNSUPPORTED;
+  // binds the device's primary context to this thread (a thread that has made no runtime
+  // call yet, such as an autograd worker, has none, and the tensor-map encoder needs it)
+  SQ_CUDA(cudaSetDevice(dev));
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& s = g_dev[dev];
   if (!s.ready) {
@@ -313,21 +314,6 @@ squad_status simt_bwd_t(const Plan& p, const BwdWs& w, uint8_t* ws, const void* 
 
 // ---------------- tensor-core backward (bf16)
 
-template <int D, int MODE, bool F32>
-squad_status launch_bwd_tc_t(DeviceState* ds, const CUtensorMap* maps, const sq::BwdArgs& a, cudaStream_t st) {
-  using Lay = sq::BwdLayout<D>;
-  auto kern = sq::squad_bwd_tc_kernel<D, MODE, F32>;
-  bool& attr = ds->bwd_attr_set[D == 128 ? 1 : 0][MODE][F32 ? 1 : 0];
-  if (!attr) {
-    SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
-    attr = true;
-  }
-  const int grid = a.total_items < ds->sms ? a.total_items : ds->sms;
-  kern<<<grid, sq::kBwdThreads, Lay::ALLOC, st>>>(maps[0], maps[1], maps[2], maps[3], a);
-  SQ_CUDA(cudaGetLastError());
-  return SQUAD_OK;
-}
-
 template <int D, bool F32>
 squad_status launch_bwd_fused_t(DeviceState* ds, const CUtensorMap* maps, const sq::BwdFusedArgs& a,
                                 cudaStream_t st) {
@@ -344,75 +330,57 @@ squad_status launch_bwd_fused_t(DeviceState* ds, const CUtensorMap* maps, const 
   return SQUAD_OK;
 }
 
-template <int MODE, bool F32>
-squad_status launch_bwd_tc(DeviceState* ds, int d, const CUtensorMap* maps, const sq::BwdArgs& a, cudaStream_t st) {
-  if (d == 128) return launch_bwd_tc_t<128, MODE, F32>(ds, maps, a, st);
-  return launch_bwd_tc_t<64, MODE, F32>(ds, maps, a, st);
-}
-
 // Backward of one pass on the tensor cores. q, k: inputs; val: the pass's values;
 // out: the pass's output; dout: its upstream gradient. f32_out selects fp32 dq/dk
 // (the global pass, whose parts are summed into the local pass's results).
 squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, const void* q, const void* k,
-                         const void* val, const void* out, const void* dout, const float* lse, float* Drow,
-                         const float* dq_add, void* dq, const float* dk_add, void* dk, __nv_bfloat16* dval,
-                         bool f32_out, cudaStream_t st) {
-  const unsigned rblocks = unsigned((p.rows + sq::kSimtWarps - 1) / sq::kSimtWarps);
-  if (d == 128)
-    sq::simt_rowdot_kernel<__nv_bfloat16, 4><<<rblocks, sq::kSimtWarps * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), Drow, p.rows, d);
-  else
-    sq::simt_rowdot_kernel<__nv_bfloat16, 2><<<rblocks, sq::kSimtWarps * 32, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), Drow, p.rows, d);
-  SQ_CUDA(cudaGetLastError());
+                         const void* val, const void* out, const void* dout, const float* lse,
+                         const float* dq_add, float* dq_acc, void* dq, const float* dk_add, void* dk,
+                         __nv_bfloat16* dval, bool f32_out, cudaStream_t st) {
   CUtensorMap maps[4];
   squad_status s;
   if ((s = encode_map(&maps[0], q, g, d, p.rows)) != SQUAD_OK) return s;
   if ((s = encode_map(&maps[1], k, g, d, p.rows)) != SQUAD_OK) return s;
   if ((s = encode_map(&maps[2], val, g, d, p.rows)) != SQUAD_OK) return s;
   if ((s = encode_map(&maps[3], dout, g, d, p.rows)) != SQUAD_OK) return s;
+  // one kernel: every (query box, key box) block once; dk and dval complete per key box
+  sq::BwdFusedArgs f{};
+  f.g = g;
+  f.total_items = g.bh * g.probs * g.nt;
+  f.scale = p.scale;
+  f.scale_log2 = p.scale * 1.4426950408889634f;
+  f.lse = lse;
+  f.out = static_cast<const __nv_bfloat16*>(out);
+  f.dout = static_cast<const __nv_bfloat16*>(dout);
+  f.add_k = dk_add;
+  f.out_k = dk;
+  f.out_val = dval;
+  f.err = ds->err;
+  f.timeout_ns = kWaitTimeoutNs;
+  const size_t n_el = size_t(p.rows) * d;
   if (g.nt == 1) {
-    // every problem is one box: one kernel computes dq, dk and dval from one S and one dP
-    sq::BwdFusedArgs f{};
-    f.g = g;
-    f.total_items = g.bh * g.probs;
-    f.scale = p.scale;
-    f.scale_log2 = p.scale * 1.4426950408889634f;
-    f.lse = lse;
-    f.Drow = Drow;
-    f.add_q = dq_add;
-    f.add_k = dk_add;
+    f.add_q = dq_add;  // dq = part (+ add), stored directly
     f.out_q = dq;
-    f.out_k = dk;
-    f.out_val = dval;
-    f.err = ds->err;
-    f.timeout_ns = kWaitTimeoutNs;
-    if (d == 128)
-      return f32_out ? launch_bwd_fused_t<128, true>(ds, maps, f, st) : launch_bwd_fused_t<128, false>(ds, maps, f, st);
-    return f32_out ? launch_bwd_fused_t<64, true>(ds, maps, f, st) : launch_bwd_fused_t<64, false>(ds, maps, f, st);
+  } else if (f32_out) {
+    // dq (fp32) = add + sum of the parts of every key box
+    f.acc_q = static_cast<float*>(dq);
+    if (dq_add != nullptr)
+      SQ_CUDA(cudaMemcpyAsync(dq, dq_add, n_el * sizeof(float), cudaMemcpyDeviceToDevice, st));
+    else
+      SQ_CUDA(cudaMemsetAsync(dq, 0, n_el * sizeof(float), st));
+  } else {
+    // dq (bf16) = bf16(add + sum of the parts): the parts are added into the fp32 addend
+    if (dq_acc == nullptr) return SQUAD_ERR_INVALID_ARG;
+    f.acc_q = dq_acc;
   }
-  sq::BwdArgs a{};
-  a.g = g;
-  a.total_items = g.bh * g.probs * g.nt;
-  a.scale = p.scale;
-  a.scale_log2 = p.scale * 1.4426950408889634f;
-  a.lse = lse;
-  a.Drow = Drow;
-  a.err = ds->err;
-  a.timeout_ns = kWaitTimeoutNs;
-  // dq
-  a.add = dq_add;
-  a.out_main = dq;
-  a.out_val = nullptr;
-  s = f32_out ? launch_bwd_tc<sq::MODE_DQ, true>(ds, d, maps, a, st)
-              : launch_bwd_tc<sq::MODE_DQ, false>(ds, d, maps, a, st);
-  if (s != SQUAD_OK) return s;
-  // dk, dval
-  a.add = dk_add;
-  a.out_main = dk;
-  a.out_val = dval;
-  return f32_out ? launch_bwd_tc<sq::MODE_DKDV, true>(ds, d, maps, a, st)
-                 : launch_bwd_tc<sq::MODE_DKDV, false>(ds, d, maps, a, st);
+  squad_status s2 =
+      d == 128 ? (f32_out ? launch_bwd_fused_t<128, true>(ds, maps, f, st) : launch_bwd_fused_t<128, false>(ds, maps, f, st))
+               : (f32_out ? launch_bwd_fused_t<64, true>(ds, maps, f, st) : launch_bwd_fused_t<64, false>(ds, maps, f, st));
+  if (s2 != SQUAD_OK || g.nt == 1 || f32_out) return s2;
+  const unsigned cblocks = unsigned((n_el / 8 + 255) / 256);
+  sq::f32_to_bf16_kernel<<<cblocks, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n_el / 8);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
 }
 
 squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k,
@@ -421,14 +389,12 @@ squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws,
   auto* dO1 = reinterpret_cast<__nv_bfloat16*>(ws + w.do1);
   float* dQ2 = reinterpret_cast<float*>(ws + w.dq2);
   float* dK2 = reinterpret_cast<float*>(ws + w.dk2);
-  float* D2 = reinterpret_cast<float*>(ws + w.D2);
-  float* D1 = reinterpret_cast<float*>(ws + w.D1);
   squad_status s;
   // global pass: values O1, output O, upstream dout -> dQ2, dK2 (fp32) and dO1
-  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, D2, nullptr, dQ2, nullptr, dK2, dO1, true, st);
+  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, nullptr, nullptr, dQ2, nullptr, dK2, dO1, true, st);
   if (s != SQUAD_OK) return s;
   // local pass: values V, output O1, upstream dO1 -> dq = dq1 + dQ2, dk = dk1 + dK2, dv
-  return tc_pass_bwd(ds, p, d, p.g1, q, k, v, o1, dO1, lse1, D1, dQ2, dq, dK2, dk,
+  return tc_pass_bwd(ds, p, d, p.g1, q, k, v, o1, dO1, lse1, dQ2, dQ2, dq, dK2, dk,
                      static_cast<__nv_bfloat16*>(dv), false, st);
 }
 
@@ -569,6 +535,9 @@ squad_status noalloc_scratch(void** out) {
   int dev = 0;
   SQ_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= kMaxDevices) return SQUAD_ERR_UNSUPPORTED;
+  // binds the device's primary context to this thread (a thread that has made no runtime
+  // call yet, such as an autograd worker, has none, and the tensor-map encoder needs it)
+  SQ_CUDA(cudaSetDevice(dev));
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (g_noalloc_ptr[dev] == nullptr) {
     void* p = nullptr;

@@ -1,30 +1,36 @@
-// squad_bwd_fused.cuh - backward of one SQuad-Attention pass whose problems fit one
-// 128-row box, in one kernel on the sm_100a tensor cores.
+// squad_bwd_fused.cuh - backward of one SQuad-Attention pass in one kernel on the
+// sm_100a tensor cores.
 //
 // The pass is softmax attention over independent problems ("SQuad: Sub-Quadratic
 // Attention Distillation for Efficient Video Generation", gist.science technical
-// summary, Methodology section 1: the groups of the global pass, and the windows of
-// the local pass when a window has at most 128 tokens). Its gradient is the textbook
-// one:
+// summary, Methodology section 1: the windows of the local pass, the groups of the
+// global pass). Its gradient is the textbook one:
 //   P = exp(s*Q K^T - lse),  dP = dO Val^T,  D = rowsum(dO o O),  dS = P o (dP - D)
 //   dVal = P^T dO,  dK = s * dS^T Q,  dQ = s * dS K.
-// When a problem is a single box, one CTA item holds the problem's Q, K, Val and dO
-// and computes all three gradients from ONE S and ONE dP: five 128-row GEMMs and one
-// read of each input, where the split dq / dk-dv kernels take seven and read twice.
+// D of a query row is computed where it is used, by the softmax thread that publishes
+// that row's statistics (two L2-resident row reads per block).
+// A problem of L tokens is cut into nt boxes of at most 128 rows. A CTA item is
+// (problem, key box kb): K_kb and Val_kb stay, the query boxes (Q_qb, dO_qb) stream,
+// and every (qb, kb) block is done once, with five GEMMs and no recomputation:
 //
-//   S^T = K Q^T   -> TMEM [0,128)    lane = key row
-//   dP^T = Val dO^T -> TMEM [128,256)
+//   S^T = K Q^T      -> TMEM [0,128)    lane = key row
+//   dP^T = Val dO^T  -> TMEM [128,256)
 //   softmax warps: P^T (bf16, in place in TMEM [0,64)) and dS^T (bf16, to shared memory)
-//   dQ  = dS K    (A = dS^T tile read MN-major)      -> TMEM [128,256)
-//   dVal = P^T dO (A = P^T from TMEM)                -> TMEM [256,384)
-//   dK  = dS^T Q  (A = dS^T tile read K-major)       -> TMEM [384,512)
+//   dQ_qb part = dS K  (A = dS^T tile read MN-major)   -> TMEM [128,256)
+//   dVal_kb += P^T dO  (A = P^T from TMEM)             -> TMEM [256,384)
+//   dK_kb  += dS^T Q   (A = dS^T tile read K-major)    -> TMEM [384,512)
+//
+// dVal and dK of a key box are complete when its item ends. dQ of a query box is
+// complete in one block when nt == 1 (stored, plus an optional fp32 addend); for
+// nt > 1 each block adds its part into an fp32 buffer with vector reductions
+// (red.global.add.v4.f32) and the host converts that buffer afterwards.
 //
 // Warp roles: warps 0-3 softmax gradient (thread = key row = TMEM lane), warps 4-7
 // epilogue (thread = token row; stores pass through a per-warp transpose patch so that
-// each warp store writes whole lines), warp 8 TMA producer, warp 9 MMA issuer.
-// Input tiles live in a pool of five slots: the next item's K and Q go into the spare
-// slot and the slot Val leaves when dP is done, so the next S can start while the
-// current item's gradients are still accumulating. Every wait is bounded.
+// each warp instruction writes whole lines), warp 8 TMA producer, warp 9 MMA issuer.
+// Input tiles live in a pool of five slots handed out in the order they are freed, so
+// the next block's Q (and, at an item boundary, K) load while the current block's
+// gradients are still accumulating. Every wait is bounded.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -34,15 +40,17 @@
 namespace sq {
 
 struct BwdFusedArgs {
-  Geom g;                  // the pass's geometry; g.nt == 1
-  int total_items;         // problems
+  Geom g;                  // the pass's geometry
+  int total_items;         // problems * nt
   float scale;             // softmax scale
   float scale_log2;        // scale * log2(e)
   const float* lse;        // [rows] natural-log LSE of this pass
-  const float* Drow;       // [rows] rowsum(dO o O) of this pass
-  const float* add_q;      // fp32 [rows, D] added to dQ, or nullptr
+  const __nv_bfloat16* out;   // [rows, D] output of this pass (for D = rowsum(dO o O))
+  const __nv_bfloat16* dout;  // [rows, D] its upstream gradient
+  const float* add_q;      // nt == 1: fp32 [rows, D] added to dQ, or nullptr
+  float* acc_q;            // nt > 1: fp32 [rows, D] that the dQ parts are added into
   const float* add_k;      // fp32 [rows, D] added to dK, or nullptr
-  void* out_q;             // dQ: fp32 if OUT_F32 else bf16
+  void* out_q;             // nt == 1: dQ, fp32 if OUT_F32 else bf16
   void* out_k;             // dK: fp32 if OUT_F32 else bf16
   __nv_bfloat16* out_val;  // dVal, bf16
   int* err;
@@ -67,70 +75,172 @@ struct BwdFusedLayout {
   static constexpr int TMEM_COLS = 512;
 };
 
-enum { G_FULL = 0, G_EMPTY = 5, G_SFULL = 10, G_PFULL, G_DQDONE, G_ACC, G_DQFREE, G_ACCFREE, G_VEC, G_DRAIN };
+enum {
+  G_FULL = 0, G_EMPTY = 5,
+  G_SFULL = 10,   // per block: S^T and dP^T are in TMEM
+  G_PFULL,        // per block: P^T and dS^T written (128 softmax threads)
+  G_DQDONE,       // per block: the dQ part is in TMEM
+  G_STEPACC,      // per block: dVal and dK MMAs done (P^T and dS^T consumed)
+  G_ITEMACC,      // per item: dVal and dK complete
+  G_DQFREE,       // per block: the epilogue drained the dQ part (128 threads)
+  G_ACCFREE,      // per item: the epilogue drained dVal and dK (128 threads)
+  G_VEC,          // per block: column statistics published (128 softmax threads)
+  G_DRAIN
+};
 
-// Slot roles of one item. After each item: the spare takes K, Val's slot (free once
-// dP is done) takes Q, K's and Q's slots take Val and dO, dO's slot becomes the spare.
-struct SlotRoles {
-  int k = 0, q = 1, v = 2, o = 3, sp = 4;
-  __device__ __forceinline__ void next() {
-    const int nk = sp, nq = v, nv = k, no = q, nsp = o;
-    k = nk;
-    q = nq;
-    v = nv;
-    o = no;
-    sp = nsp;
+// Tile slots of the blocks, identical on the producer and the MMA issuer. Slots are
+// handed out first-freed first-used: the five free slots, then the releases of the
+// blocks in order (Val after the item's last dP; Q, dO after each block's
+// accumulation; K after the item's last one). A release is taken into the queue only
+// when the queue runs dry, which fixes the order independently of timing.
+struct SlotPlan {
+  struct Rec {
+    int k, v, q, o;
+    bool last;
+  };
+  uint32_t fifo = 0x43210u;  // 4 bits per free slot, front in the low bits
+  int n = 5;
+  Rec rec[4];
+  int head = 0, tail = 0;  // blocks whose releases are not yet queued: [head, tail)
+  int ck = 0, cv = 0;
+  __device__ __forceinline__ void push(int s) {
+    fifo |= uint32_t(s) << (4 * n);
+    ++n;
+  }
+  __device__ __forceinline__ int pop() {
+    while (n == 0 && head < tail) {
+      const Rec& r = rec[head & 3];
+      if (r.last) push(r.v);
+      push(r.q);
+      push(r.o);
+      if (r.last) push(r.k);
+      ++head;
+    }
+    const int s = int(fifo & 15u);
+    fifo >>= 4;
+    --n;
+    return s;
+  }
+  // slots of the next block: all four tiles at an item's first block, Q and dO after
+  __device__ __forceinline__ Rec next(bool first, bool last) {
+    Rec r;
+    if (first) {
+      r.k = pop();
+      r.q = pop();
+      r.v = pop();
+      r.o = pop();
+      ck = r.k;
+      cv = r.v;
+    } else {
+      r.k = ck;
+      r.v = cv;
+      r.q = pop();
+      r.o = pop();
+    }
+    r.last = last;
+    rec[tail & 3] = r;
+    ++tail;
+    return r;
   }
 };
 
-// Epilogue of one fp32 accumulator (thread = row): out = acc * scale (+ add), written
-// as fp32 or bf16 rows through the warp's 128B-swizzled patch, 32 columns per round.
-template <int D, bool OUT_F32>
-__device__ __forceinline__ void epi_rows_f32(uint32_t taddr, uint32_t xp, int lane, size_t tok, bool live,
-                                             float scale, const float* add, void* out) {
+// D of one row: sum over d of dO[d] * O[d], bf16 rows widened exactly, fp32 sum.
+template <int D>
+__device__ __forceinline__ float row_dot(const __nv_bfloat16* a, const __nv_bfloat16* b) {
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  const uint4* b4 = reinterpret_cast<const uint4*>(b);
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int j = 0; j < D / 8; ++j) {
+    const uint4 x = __ldg(a4 + j), y = __ldg(b4 + j);
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc0 = fmaf(__uint_as_float(xs[u] << 16), __uint_as_float(ys[u] << 16), acc0);
+      acc1 = fmaf(__uint_as_float(xs[u] & 0xffff0000u), __uint_as_float(ys[u] & 0xffff0000u), acc1);
+    }
+  }
+  return acc0 + acc1;
+}
+
+// Rows an epilogue lane writes: a warp drains its 32 TMEM lanes (one row each) through
+// a 128B-swizzled patch and writes them back four rows per instruction; lane l handles
+// rows 4i + l/8 (i < 8), 16-byte column chunk l%8. Token rows are shuffled once per box.
+struct EpiRows {
+  int tok[8];
+  uint32_t live;  // bit r: warp row r is inside the problem
+};
+
+__device__ __forceinline__ EpiRows epi_rows_of(int lane, int my_tok, bool my_live) {
+  EpiRows e;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) e.tok[i] = __shfl_sync(0xffffffffu, my_tok, 4 * i + (lane >> 3));
+  e.live = __ballot_sync(0xffffffffu, my_live);
+  return e;
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_RED = 2 };
+
+// Drain one fp32 accumulator (D columns): value = acc * scale (+ add), then stored as
+// fp32 (EPI_F32) or bf16 (EPI_BF16), or added into fp32 memory (EPI_RED). 64 columns at
+// a time: the addend loads are issued before the TMEM load so their latencies overlap.
+template <int D, int KIND>
+__device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, const EpiRows& R, float scale,
+                                        const float* add, void* out) {
   const int lr = lane >> 3, lc = lane & 7;
 #pragma unroll 1
-  for (int rd = 0; rd < D / 32; ++rd) {
-    uint32_t v[32];
-    tmem_ld32(taddr + rd * 32, v);
+  for (int h = 0; h < D / 64; ++h) {
+    float4 a[2][8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * c]) * scale),
-                   __float_as_uint(__uint_as_float(v[4 * c + 1]) * scale),
-                   __float_as_uint(__uint_as_float(v[4 * c + 2]) * scale),
-                   __float_as_uint(__uint_as_float(v[4 * c + 3]) * scale));
-    __syncwarp();
+    for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = 4 * i + lr;
-      const size_t rtok = __shfl_sync(0xffffffffu, tok, r);
-      const bool rlive = __shfl_sync(0xffffffffu, live, r);
-      const uint4 x = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
-      if (rlive) {
-        float4 f = make_float4(__uint_as_float(x.x), __uint_as_float(x.y), __uint_as_float(x.z), __uint_as_float(x.w));
-        const size_t e = rtok * D + rd * 32 + lc * 4;
-        if (add != nullptr) {
-          const float4 a = *reinterpret_cast<const float4*>(add + e);
-          f.x += a.x;
-          f.y += a.y;
-          f.z += a.z;
-          f.w += a.w;
-        }
-        if (OUT_F32)
-          *reinterpret_cast<float4*>(static_cast<float*>(out) + e) = f;
-        else
-          *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + e) =
-              make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+      for (int i = 0; i < 8; ++i) {
+        a[rr][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (add != nullptr && ((R.live >> (4 * i + lr)) & 1u))
+          a[rr][i] = __ldg(reinterpret_cast<const float4*>(add + size_t(R.tok[i]) * D + h * 64 + rr * 32 + lc * 4));
       }
+    uint32_t v[64];
+    tmem_ld64(taddr + h * 64, v);
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4),
+                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c]) * scale),
+                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 1]) * scale),
+                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 2]) * scale),
+                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 3]) * scale));
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + lr;
+        const uint4 x = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
+        if ((R.live >> r) & 1u) {
+          const float f0 = __uint_as_float(x.x) + a[rr][i].x, f1 = __uint_as_float(x.y) + a[rr][i].y;
+          const float f2 = __uint_as_float(x.z) + a[rr][i].z, f3 = __uint_as_float(x.w) + a[rr][i].w;
+          const size_t e = size_t(R.tok[i]) * D + h * 64 + rr * 32 + lc * 4;
+          if (KIND == EPI_F32)
+            *reinterpret_cast<float4*>(static_cast<float*>(out) + e) = make_float4(f0, f1, f2, f3);
+          else if (KIND == EPI_BF16)
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + e) =
+                make_uint2(pack_bf16x2(f0, f1), pack_bf16x2(f2, f3));
+          else
+            red_add_v4(static_cast<float*>(out) + e, f0, f1, f2, f3);
+        }
+      }
+      __syncwarp();
     }
-    __syncwarp();
   }
 }
 
-// Epilogue of one fp32 accumulator written as bf16 rows, 64 columns per round.
+// Drain one fp32 accumulator as bf16 rows (no scale), 64 columns per round.
 template <int D>
-__device__ __forceinline__ void epi_rows_bf16(uint32_t taddr, uint32_t xp, int lane, size_t tok, bool live,
-                                              __nv_bfloat16* out) {
+__device__ __forceinline__ void epi_acc_bf16(uint32_t taddr, uint32_t xp, int lane, const EpiRows& R,
+                                             __nv_bfloat16* out) {
   const int lr = lane >> 3, lc = lane & 7;
 #pragma unroll 1
   for (int h = 0; h < D / 64; ++h) {
@@ -147,13 +257,21 @@ __device__ __forceinline__ void epi_rows_bf16(uint32_t taddr, uint32_t xp, int l
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = 4 * i + lr;
-      const size_t rtok = __shfl_sync(0xffffffffu, tok, r);
-      const bool rlive = __shfl_sync(0xffffffffu, live, r);
       const uint4 x = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
-      if (rlive) *reinterpret_cast<uint4*>(out + rtok * D + h * 64 + lc * 8) = x;
+      if ((R.live >> r) & 1u) *reinterpret_cast<uint4*>(out + size_t(R.tok[i]) * D + h * 64 + lc * 8) = x;
     }
     __syncwarp();
   }
+}
+
+// dq = bf16(acc), 8 elements per thread (rows * d is a multiple of 8)
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out, size_t n8) {
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(in)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(in)[2 * i + 1];
+  reinterpret_cast<uint4*>(out)[i] =
+      make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
 template <int D, bool OUT_F32>
@@ -188,7 +306,8 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     mbar_init(&bars[G_SFULL], 1);
     mbar_init(&bars[G_PFULL], 128);
     mbar_init(&bars[G_DQDONE], 1);
-    mbar_init(&bars[G_ACC], 1);
+    mbar_init(&bars[G_STEPACC], 1);
+    mbar_init(&bars[G_ITEMACC], 1);
     mbar_init(&bars[G_DQFREE], 128);
     mbar_init(&bars[G_ACCFREE], 128);
     mbar_init(&bars[G_VEC], 128);
@@ -214,16 +333,18 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   auto slot_addr = [&](int s) -> uint32_t { return sbase + Lay::SLOT_OFF + s * Lay::TILE; };
 
+  const int nt = g.nt;
+
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      SlotRoles R;
+      SlotPlan plan;
       uint32_t pu = 0, used = 0;  // per slot: parity of its use count; ever used
       const uint32_t tx = uint32_t(g.box_rows) * D * 2;
-      int b0, c0;
-      tile_origin(g, 0, b0, c0);
-      auto load = [&](int s, const CUtensorMap* m, int base) -> bool {
+      auto load = [&](int s, const CUtensorMap* m, int base, int t) -> bool {
         if (!mbar_wait(&bars[G_EMPTY + s], ((pu >> s) & 1u) ^ 1u, abort_flag, to)) return false;
+        int b0, c0;
+        tile_origin(g, t, b0, c0);
         mbar_arrive_expect_tx(&bars[G_FULL + s], tx);
 #pragma unroll
         for (int dh = 0; dh < DH; ++dh)
@@ -233,13 +354,20 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         used |= 1u << s;
         return true;
       };
-      for (int item = blockIdx.x; item < args.total_items; item += gridDim.x) {
-        const int base = problem_base(g, item);
-        // K and Q first: they go to slots that free early, so the next S can start soon
-        if (!(load(R.k, &tm_k, base) && load(R.q, &tm_q, base) && load(R.v, &tm_v, base) &&
-              load(R.o, &tm_do, base)))
-          break;
-        R.next();
+      bool ok = true;
+      for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
+        const int prob = item / nt, kb = item - prob * nt;
+        const int base = problem_base(g, prob);
+        for (int qb = 0; qb < nt; ++qb) {
+          const SlotPlan::Rec r = plan.next(qb == 0, qb == nt - 1);
+          // K and Q first: S needs only them
+          if (qb == 0)
+            ok = load(r.k, &tm_k, base, kb) && load(r.q, &tm_q, base, qb) && load(r.v, &tm_v, base, kb) &&
+                 load(r.o, &tm_do, base, qb);
+          else
+            ok = load(r.q, &tm_q, base, qb) && load(r.o, &tm_do, base, qb);
+          if (!ok) break;
+        }
       }
       for (int s = 0; s < Lay::NSLOT; ++s)
         if ((used >> s) & 1u) mbar_wait_drain(&bars[G_FULL + s], ((pu >> s) & 1u) ^ 1u, to);
@@ -247,68 +375,78 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      SlotRoles R;
-      uint32_t cu = 0, i = 0;
+      SlotPlan plan;
+      uint32_t cu = 0, i = 0, t = 0;  // consumer parities; item and block counters
       const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);   // S^T, dP^T: both operands K-major
       const uint32_t id_kv = idesc_bf16_f32(128, D, 0, 1);    // dVal, dK: B MN-major
       const uint32_t id_q = idesc_bf16_f32(128, D, 1, 1);     // dQ: A (dS^T tile) and B MN-major
       const uint32_t ds = sbase + Lay::DS_OFF;
       bool ok = true;
       auto wait_full = [&](int s) -> bool {
-        return mbar_wait(&bars[G_FULL + s], (cu >> s) & 1u, abort_flag, to);
+        const bool r = mbar_wait(&bars[G_FULL + s], (cu >> s) & 1u, abort_flag, to);
+        cu ^= 1u << s;
+        return r;
       };
-      for (int item = blockIdx.x; item < args.total_items; item += gridDim.x, ++i) {
-        const uint32_t sk = slot_addr(R.k), sq_ = slot_addr(R.q), sv = slot_addr(R.v), so = slot_addr(R.o);
-        // S^T into [0,128): the previous dVal has read P^T from there
-        if (i > 0) ok = mbar_wait(&bars[G_ACC], (i - 1) & 1u, abort_flag, to);
-        ok = ok && wait_full(R.k) && wait_full(R.q);
-        if (!ok) break;
-        tc_fence_after();
+      for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x, ++i) {
+        for (int qb = 0; qb < nt; ++qb, ++t) {
+          const bool first = qb == 0, last = qb == nt - 1;
+          const SlotPlan::Rec r = plan.next(first, last);
+          const uint32_t sk = slot_addr(r.k), sq_ = slot_addr(r.q), sv = slot_addr(r.v), so = slot_addr(r.o);
+          // S^T into [0,128): the previous block's dVal has read P^T from there
+          if (t > 0) ok = mbar_wait(&bars[G_STEPACC], (t - 1) & 1u, abort_flag, to);
+          if (ok && first) ok = wait_full(r.k);
+          ok = ok && wait_full(r.q);
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-          mma_ss(tmem + Lay::TM_S, sdesc_sw128(sk + koff, 16, 1024), sdesc_sw128(sq_ + koff, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+            mma_ss(tmem + Lay::TM_S, sdesc_sw128(sk + koff, 16, 1024), sdesc_sw128(sq_ + koff, 16, 1024), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          // dP^T into [128,256): the epilogue has drained the previous dQ part from there
+          if (t > 0) ok = mbar_wait(&bars[G_DQFREE], (t - 1) & 1u, abort_flag, to);
+          if (ok && first) ok = wait_full(r.v);
+          ok = ok && wait_full(r.o);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
+            mma_ss(tmem + Lay::TM_DP, sdesc_sw128(sv + koff, 16, 1024), sdesc_sw128(so + koff, 16, 1024), id_s,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[G_SFULL]);
+          if (last) tc_commit(&bars[G_EMPTY + r.v]);  // Val is done
+          if (!(ok = mbar_wait(&bars[G_PFULL], t & 1u, abort_flag, to))) break;
+          tc_fence_after();
+          // dQ part = dS K (K = key rows): A = dS^T tile (rows = keys, query-contiguous: MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + Lay::TM_DP, sdesc_sw128(ds + kk * 2048, BLK, 1024), sdesc_sw128(sk + kk * 2048, BLK, 1024),
+                   id_q, kk > 0 ? 1u : 0u);
+          tc_commit(&bars[G_DQDONE]);
+          // the first block of an item overwrites dVal and dK: the epilogue has drained the last item's
+          if (first && i > 0 && !(ok = mbar_wait(&bars[G_ACCFREE], (i - 1) & 1u, abort_flag, to))) break;
+          tc_fence_after();
+          // dVal += P^T dO (K = query rows): A = P^T in TMEM columns [0,64)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + Lay::TM_DV, tmem + Lay::TM_S + kk * 8, sdesc_sw128(so + kk * 2048, BLK, 1024), id_kv,
+                   (!first || kk > 0) ? 1u : 0u);
+          // dK += dS^T Q (K = query rows): A = dS^T tile, K-major
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + Lay::TM_DK, sdesc_sw128(ds + (kk >> 2) * BLK + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(sq_ + kk * 2048, BLK, 1024), id_kv, (!first || kk > 0) ? 1u : 0u);
+          tc_commit(&bars[G_STEPACC]);
+          tc_commit(&bars[G_EMPTY + r.q]);
+          tc_commit(&bars[G_EMPTY + r.o]);
+          if (last) {
+            tc_commit(&bars[G_EMPTY + r.k]);
+            tc_commit(&bars[G_ITEMACC]);
+          }
         }
-        // dP^T into [128,256): the epilogue has drained the previous dQ from there
-        if (i > 0) ok = mbar_wait(&bars[G_DQFREE], (i - 1) & 1u, abort_flag, to);
-        ok = ok && wait_full(R.v) && wait_full(R.o);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk >> 2) * BLK + (kk & 3) * 32;
-          mma_ss(tmem + Lay::TM_DP, sdesc_sw128(sv + koff, 16, 1024), sdesc_sw128(so + koff, 16, 1024), id_s,
-                 kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars[G_SFULL]);
-        tc_commit(&bars[G_EMPTY + R.v]);  // Val is done
-        cu ^= (1u << R.k) | (1u << R.q) | (1u << R.v) | (1u << R.o);
-        if (!(ok = mbar_wait(&bars[G_PFULL], i & 1u, abort_flag, to))) break;
-        tc_fence_after();
-        // dQ = dS K (K = key rows): A = dS^T tile (rows = keys, query-contiguous: MN-major)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + Lay::TM_DP, sdesc_sw128(ds + kk * 2048, BLK, 1024), sdesc_sw128(sk + kk * 2048, BLK, 1024),
-                 id_q, kk > 0 ? 1u : 0u);
-        tc_commit(&bars[G_DQDONE]);
-        if (i > 0 && !(ok = mbar_wait(&bars[G_ACCFREE], (i - 1) & 1u, abort_flag, to))) break;
-        tc_fence_after();
-        // dVal = P^T dO (K = query rows): A = P^T in TMEM columns [0,64)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + Lay::TM_DV, tmem + Lay::TM_S + kk * 8, sdesc_sw128(so + kk * 2048, BLK, 1024), id_kv,
-                 kk > 0 ? 1u : 0u);
-        // dK = dS^T Q (K = query rows): A = dS^T tile, K-major
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + Lay::TM_DK, sdesc_sw128(ds + (kk >> 2) * BLK + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(sq_ + kk * 2048, BLK, 1024), id_kv, kk > 0 ? 1u : 0u);
-        tc_commit(&bars[G_ACC]);
-        tc_commit(&bars[G_EMPTY + R.k]);
-        tc_commit(&bars[G_EMPTY + R.q]);
-        tc_commit(&bars[G_EMPTY + R.o]);
-        R.next();
       }
       tc_commit(&bars[G_DRAIN]);
       mbar_wait_drain(&bars[G_DRAIN], 0, to);
@@ -321,65 +459,68 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     const uint32_t ds_row = sbase + Lay::DS_OFF + row * 128;
     const float c2 = args.scale_log2;
     const float log2e = 1.4426950408889634f;
-    const int valid = tile_valid_rows(g, 0);
-    const bool rlive = row < valid;
-    const int roff = rlive ? tile_row_offset(g, 0, row) : 0;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
-    uint32_t i = 0;
-    for (int item = blockIdx.x; item < args.total_items; item += gridDim.x, ++i) {
-      // per-query statistics (the query box is the key box): row r publishes column r
-      float* vl = vec + (i & 1u) * 256;
-      float l = INFINITY, dd = 0.f;  // query columns past the problem: P = 0
-      if (rlive) {
-        const int tok = problem_base(g, item) + roff;
-        l = args.lse[tok] * log2e;
-        dd = args.Drow[tok];
-      }
-      vl[row] = l;
-      vl[128 + row] = dd;
-      mbar_arrive(&bars[G_VEC]);
-      if (!wwait(&bars[G_VEC], i & 1u)) break;
-      if (!wwait(&bars[G_SFULL], i & 1u)) break;
-      tc_fence_after();
+    uint32_t t = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
+      const int prob = item / nt, kb = item - prob * nt;
+      const int base = problem_base(g, prob);
+      const bool rlive = row < tile_valid_rows(g, kb);
+      for (int qb = 0; qb < nt; ++qb, ++t) {
+        // per-query statistics of the block's query box: row r publishes column r
+        float* vl = vec + (t & 1u) * 256;
+        float l = INFINITY, dd = 0.f;  // query columns past the problem: P = 0
+        if (row < tile_valid_rows(g, qb)) {
+          const int tok = base + tile_row_offset(g, qb, row);
+          l = args.lse[tok] * log2e;
+          dd = row_dot<D>(args.dout + size_t(tok) * D, args.out + size_t(tok) * D);
+        }
+        vl[row] = l;
+        vl[128 + row] = dd;
+        mbar_arrive(&bars[G_VEC]);
+        if (!(ok = wwait(&bars[G_VEC], t & 1u))) break;
+        if (!(ok = wwait(&bars[G_SFULL], t & 1u))) break;
+        tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32], dp[32];
-        tmem_ld32(tS + c * 32, s);
-        tmem_ld32(tDP + c * 32, dp);
-        uint32_t pk[16], dk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], dp[32];
+          tmem_ld32(tS + c * 32, s);
+          tmem_ld32(tDP + c * 32, dp);
+          uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int e4 = 0; e4 < 32; e4 += 4) {
-          const float4 lc4 = *reinterpret_cast<const float4*>(vl + c * 32 + e4);
-          const float4 dc4 = *reinterpret_cast<const float4*>(vl + 128 + c * 32 + e4);
-          const float lcol[4] = {lc4.x, lc4.y, lc4.z, lc4.w};
-          const float dcol[4] = {dc4.x, dc4.y, dc4.z, dc4.w};
-          float p[4], dsv[4];
+          for (int e4 = 0; e4 < 32; e4 += 4) {
+            const float4 lc4 = *reinterpret_cast<const float4*>(vl + c * 32 + e4);
+            const float4 dc4 = *reinterpret_cast<const float4*>(vl + 128 + c * 32 + e4);
+            const float lcol[4] = {lc4.x, lc4.y, lc4.z, lc4.w};
+            const float dcol[4] = {dc4.x, dc4.y, dc4.z, dc4.w};
+            float p[4], dsv[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            // key rows past the problem: P = dS = 0 (a select: exp2 of a zero score may overflow)
-            p[u] = rlive ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
-            dsv[u] = p[u] * (__uint_as_float(dp[e4 + u]) - dcol[u]);
+            for (int u = 0; u < 4; ++u) {
+              // key rows past the problem: P = dS = 0 (a select: exp2 of a zero score may overflow)
+              p[u] = rlive ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
+              dsv[u] = p[u] * (__uint_as_float(dp[e4 + u]) - dcol[u]);
+            }
+            pk[e4 >> 1] = pack_bf16x2(p[0], p[1]);
+            pk[(e4 >> 1) + 1] = pack_bf16x2(p[2], p[3]);
+            dk[e4 >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            dk[(e4 >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
-          pk[e4 >> 1] = pack_bf16x2(p[0], p[1]);
-          pk[(e4 >> 1) + 1] = pack_bf16x2(p[2], p[3]);
-          dk[e4 >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-          dk[(e4 >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
-        }
-        tmem_st16(tS + c * 16, pk);
-        // dS^T row: query columns [32c, 32c+32) are 16-byte chunks 4(c&1)..4(c&1)+3 of block c>>1
+          tmem_st16(tS + c * 16, pk);
+          // dS^T row: query columns [32c, 32c+32) are 16-byte chunks 4(c&1)..4(c&1)+3 of block c>>1
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int chunk = (c & 1) * 4 + j;
-          st_shared_v4(ds_row + (c >> 1) * BLK + ((chunk ^ (row & 7)) << 4), dk[4 * j], dk[4 * j + 1], dk[4 * j + 2],
-                       dk[4 * j + 3]);
+          for (int j = 0; j < 4; ++j) {
+            const int chunk = (c & 1) * 4 + j;
+            st_shared_v4(ds_row + (c >> 1) * BLK + ((chunk ^ (row & 7)) << 4), dk[4 * j], dk[4 * j + 1],
+                         dk[4 * j + 2], dk[4 * j + 3]);
+          }
         }
+        tmem_st_wait();
+        fence_async_smem();  // the dS^T tile is read by the tensor core
+        tc_fence_before();
+        mbar_arrive(&bars[G_PFULL]);
       }
-      tmem_st_wait();
-      fence_async_smem();  // the dS^T tile is read by the tensor core
-      tc_fence_before();
-      mbar_arrive(&bars[G_PFULL]);
     }
   } else {
     // ------------------------------------------------------------ epilogue (thread = token row)
@@ -387,26 +528,35 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     const int row = q4 * 32 + lane;
     const uint32_t lane_sel = uint32_t(q4 * 32) << 16;
     const uint32_t xp = sbase + Lay::XP_OFF + q4 * 4096;
-    const int valid = tile_valid_rows(g, 0);
-    const bool live = row < valid;
-    const int roff = live ? tile_row_offset(g, 0, row) : 0;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
-    uint32_t i = 0;
-    for (int item = blockIdx.x; item < args.total_items; item += gridDim.x, ++i) {
-      const size_t tok = live ? size_t(problem_base(g, item) + roff) : 0;
-      if (!wwait(&bars[G_DQDONE], i & 1u)) break;
+    uint32_t i = 0, t = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x, ++i) {
+      const int prob = item / nt, kb = item - prob * nt;
+      const int base = problem_base(g, prob);
+      for (int qb = 0; qb < nt; ++qb, ++t) {
+        const bool liveq = row < tile_valid_rows(g, qb);
+        const EpiRows RQ = epi_rows_of(lane, liveq ? base + tile_row_offset(g, qb, row) : 0, liveq);
+        if (!(ok = wwait(&bars[G_DQDONE], t & 1u))) break;
+        tc_fence_after();
+        const uint32_t tq = tmem + lane_sel + Lay::TM_DP;
+        if (nt > 1)
+          epi_acc<D, EPI_RED>(tq, xp, lane, RQ, args.scale, nullptr, args.acc_q);
+        else
+          epi_acc<D, OUT_F32 ? EPI_F32 : EPI_BF16>(tq, xp, lane, RQ, args.scale, args.add_q, args.out_q);
+        tc_fence_before();
+        mbar_arrive(&bars[G_DQFREE]);
+      }
+      if (!ok) break;
+      const bool livek = row < tile_valid_rows(g, kb);
+      const EpiRows RK = epi_rows_of(lane, livek ? base + tile_row_offset(g, kb, row) : 0, livek);
+      if (!(ok = wwait(&bars[G_ITEMACC], i & 1u))) break;
       tc_fence_after();
-      epi_rows_f32<D, OUT_F32>(tmem + lane_sel + Lay::TM_DP, xp, lane, tok, live, args.scale, args.add_q,
-                               args.out_q);
-      tc_fence_before();
-      mbar_arrive(&bars[G_DQFREE]);
-      if (!wwait(&bars[G_ACC], i & 1u)) break;
-      tc_fence_after();
-      epi_rows_bf16<D>(tmem + lane_sel + Lay::TM_DV, xp, lane, tok, live, args.out_val);
-      epi_rows_f32<D, OUT_F32>(tmem + lane_sel + Lay::TM_DK, xp, lane, tok, live, args.scale, args.add_k,
-                               args.out_k);
+      epi_acc_bf16<D>(tmem + lane_sel + Lay::TM_DV, xp, lane, RK, args.out_val);
+      epi_acc<D, OUT_F32 ? EPI_F32 : EPI_BF16>(tmem + lane_sel + Lay::TM_DK, xp, lane, RK, args.scale, args.add_k,
+                                               args.out_k);
       tc_fence_before();
       mbar_arrive(&bars[G_ACCFREE]);
     }

@@ -216,3 +216,29 @@ def test_cpu_tensors_are_rejected():
     inp = random_problem(31, 1, 1, 64, grid, tile, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         sq.squad_attn_fwd(inp.q, inp.k, inp.v, grid, tile)
+
+
+def test_call_from_a_fresh_thread(cuda_ok):
+    # a thread that has made no CUDA runtime call has no context bound; the library binds it
+    import threading
+    grid, tile = (4, 8, 8), (1, 4, 4)
+    inp = random_problem(37, 1, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    qd, kd, vd, dod = _dev(inp.q, inp.k, inp.v, inp.do)
+    torch.cuda.synchronize()
+    res = {}
+
+    def work():
+        try:
+            o, o1, l1, l2 = sq.squad_attn_fwd(qd, kd, vd, grid, tile)
+            res["grads"] = sq.squad_attn_bwd(qd, kd, vd, o, o1, l1, l2, dod, grid, tile)
+            torch.cuda.synchronize()
+        except Exception as e:  # reported on the main thread
+            res["err"] = e
+
+    th = threading.Thread(target=work)
+    th.start()
+    th.join()
+    assert "err" not in res, res.get("err")
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, a, r in zip(("dQ", "dK", "dV"), res["grads"], ref):
+        assert_close(a.cpu().double().numpy(), r, GRAD_MAX, name)

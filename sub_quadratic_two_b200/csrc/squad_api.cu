@@ -334,8 +334,8 @@ squad_status launch_bwd_fused_t(DeviceState* ds, const CUtensorMap* maps, const 
 // out: the pass's output; dout: its upstream gradient. f32_out selects fp32 dq/dk
 // (the global pass, whose parts are summed into the local pass's results).
 squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, const void* q, const void* k,
-                         const void* val, const void* out, const void* dout, const float* lse,
-                         const float* dq_add, float* dq_acc, void* dq, const float* dk_add, void* dk,
+                         const void* val, const void* out, const void* dout, const float* lse, const float* Drow,
+                         float* d_next, const float* dq_add, float* dq_acc, void* dq, const float* dk_add, void* dk,
                          __nv_bfloat16* dval, bool f32_out, cudaStream_t st) {
   CUtensorMap maps[4];
   squad_status s;
@@ -350,8 +350,11 @@ squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, c
   f.scale = p.scale;
   f.scale_log2 = p.scale * 1.4426950408889634f;
   f.lse = lse;
+  f.Drow = Drow;
   f.out = static_cast<const __nv_bfloat16*>(out);
   f.dout = static_cast<const __nv_bfloat16*>(dout);
+  f.val = static_cast<const __nv_bfloat16*>(val);
+  f.d_next = d_next;
   f.add_k = dk_add;
   f.out_k = dk;
   f.out_val = dval;
@@ -389,12 +392,15 @@ squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws,
   auto* dO1 = reinterpret_cast<__nv_bfloat16*>(ws + w.do1);
   float* dQ2 = reinterpret_cast<float*>(ws + w.dq2);
   float* dK2 = reinterpret_cast<float*>(ws + w.dk2);
+  float* D1 = reinterpret_cast<float*>(ws + w.D1);
   squad_status s;
-  // global pass: values O1, output O, upstream dout -> dQ2, dK2 (fp32) and dO1
-  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, nullptr, nullptr, dQ2, nullptr, dK2, dO1, true, st);
+  // global pass: values O1, output O, upstream dout -> dQ2, dK2 (fp32), dO1 and the
+  // local pass's D1 = rowsum(dO1 o O1); its own D is computed in the kernel
+  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, nullptr, D1, nullptr, nullptr, dQ2, nullptr, dK2, dO1,
+                  true, st);
   if (s != SQUAD_OK) return s;
   // local pass: values V, output O1, upstream dO1 -> dq = dq1 + dQ2, dk = dk1 + dK2, dv
-  return tc_pass_bwd(ds, p, d, p.g1, q, k, v, o1, dO1, lse1, dQ2, dQ2, dq, dK2, dk,
+  return tc_pass_bwd(ds, p, d, p.g1, q, k, v, o1, dO1, lse1, D1, nullptr, dQ2, dQ2, dq, dK2, dk,
                      static_cast<__nv_bfloat16*>(dv), false, st);
 }
 

@@ -7,8 +7,10 @@
 // global pass). Its gradient is the textbook one:
 //   P = exp(s*Q K^T - lse),  dP = dO Val^T,  D = rowsum(dO o O),  dS = P o (dP - D)
 //   dVal = P^T dO,  dK = s * dS^T Q,  dQ = s * dS K.
-// D of a query row is computed where it is used, by the softmax thread that publishes
-// that row's statistics (two L2-resident row reads per block).
+// D of a query row is read from a vector or computed by the softmax warps from dO and
+// O rows (four rows per load instruction). The epilogue can also produce the D of the
+// pass that made Val: rowsum(dVal o Val) over the rows it writes (the global pass
+// gives the local pass its D this way).
 // A problem of L tokens is cut into nt boxes of at most 128 rows. A CTA item is
 // (problem, key box kb): K_kb and Val_kb stay, the query boxes (Q_qb, dO_qb) stream,
 // and every (qb, kb) block is done once, with five GEMMs and no recomputation:
@@ -45,8 +47,11 @@ struct BwdFusedArgs {
   float scale;             // softmax scale
   float scale_log2;        // scale * log2(e)
   const float* lse;        // [rows] natural-log LSE of this pass
-  const __nv_bfloat16* out;   // [rows, D] output of this pass (for D = rowsum(dO o O))
-  const __nv_bfloat16* dout;  // [rows, D] its upstream gradient
+  const float* Drow;          // [rows] D = rowsum(dO o O) of this pass, or nullptr: computed here
+  const __nv_bfloat16* out;   // [rows, D] output of this pass (read when Drow == nullptr)
+  const __nv_bfloat16* dout;  // [rows, D] its upstream gradient (read when Drow == nullptr)
+  const __nv_bfloat16* val;   // [rows, D] values of this pass (read when d_next != nullptr)
+  float* d_next;              // [rows] rowsum(dVal o Val), the D of the pass that produced Val, or nullptr
   const float* add_q;      // nt == 1: fp32 [rows, D] added to dQ, or nullptr
   float* acc_q;            // nt > 1: fp32 [rows, D] that the dQ parts are added into
   const float* add_k;      // fp32 [rows, D] added to dK, or nullptr
@@ -100,8 +105,10 @@ struct SlotPlan {
   };
   uint32_t fifo = 0x43210u;  // 4 bits per free slot, front in the low bits
   int n = 5;
-  Rec rec[4];
-  int head = 0, tail = 0;  // blocks whose releases are not yet queued: [head, tail)
+  // blocks whose releases are not yet queued: [head, tail); at most two (the current block
+  // and the one before it) are ever pending, kept in r0 / r1 by parity
+  Rec r0{}, r1{};
+  int head = 0, tail = 0;
   int ck = 0, cv = 0;
   __device__ __forceinline__ void push(int s) {
     fifo |= uint32_t(s) << (4 * n);
@@ -109,7 +116,7 @@ struct SlotPlan {
   }
   __device__ __forceinline__ int pop() {
     while (n == 0 && head < tail) {
-      const Rec& r = rec[head & 3];
+      const Rec r = (head & 1) ? r1 : r0;
       if (r.last) push(r.v);
       push(r.q);
       push(r.o);
@@ -138,29 +145,24 @@ struct SlotPlan {
       r.o = pop();
     }
     r.last = last;
-    rec[tail & 3] = r;
+    if (tail & 1)
+      r1 = r;
+    else
+      r0 = r;
     ++tail;
     return r;
   }
 };
 
-// D of one row: sum over d of dO[d] * O[d], bf16 rows widened exactly, fp32 sum.
-template <int D>
-__device__ __forceinline__ float row_dot(const __nv_bfloat16* a, const __nv_bfloat16* b) {
-  const uint4* a4 = reinterpret_cast<const uint4*>(a);
-  const uint4* b4 = reinterpret_cast<const uint4*>(b);
-  float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-  for (int j = 0; j < D / 8; ++j) {
-    const uint4 x = __ldg(a4 + j), y = __ldg(b4 + j);
-    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+// Dot product of two 8-element bf16 chunks (widened exactly), added to acc.
+__device__ __forceinline__ float dot8_bf16(const uint4& x, const uint4& y, float acc) {
+  const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      acc0 = fmaf(__uint_as_float(xs[u] << 16), __uint_as_float(ys[u] << 16), acc0);
-      acc1 = fmaf(__uint_as_float(xs[u] & 0xffff0000u), __uint_as_float(ys[u] & 0xffff0000u), acc1);
-    }
+  for (int u = 0; u < 4; ++u) {
+    acc = fmaf(__uint_as_float(xs[u] << 16), __uint_as_float(ys[u] << 16), acc);
+    acc = fmaf(__uint_as_float(xs[u] & 0xffff0000u), __uint_as_float(ys[u] & 0xffff0000u), acc);
   }
-  return acc0 + acc1;
+  return acc;
 }
 
 // Rows an epilogue lane writes: a warp drains its 32 TMEM lanes (one row each) through
@@ -186,8 +188,8 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_RED = 2 };
 
 // Drain one fp32 accumulator (D columns): value = acc * scale (+ add), then stored as
-// fp32 (EPI_F32) or bf16 (EPI_BF16), or added into fp32 memory (EPI_RED). 64 columns at
-// a time: the addend loads are issued before the TMEM load so their latencies overlap.
+// fp32 (EPI_F32) or bf16 (EPI_BF16), or added into fp32 memory (EPI_RED). The addend
+// loads of 64 columns are issued before their TMEM loads so the latencies overlap.
 template <int D, int KIND>
 __device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, const EpiRows& R, float scale,
                                         const float* add, void* out) {
@@ -203,17 +205,16 @@ __device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, c
         if (add != nullptr && ((R.live >> (4 * i + lr)) & 1u))
           a[rr][i] = __ldg(reinterpret_cast<const float4*>(add + size_t(R.tok[i]) * D + h * 64 + rr * 32 + lc * 4));
       }
-    uint32_t v[64];
-    tmem_ld64(taddr + h * 64, v);
 #pragma unroll
     for (int rr = 0; rr < 2; ++rr) {
+      uint32_t v[32];
+      tmem_ld32(taddr + h * 64 + rr * 32, v);
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4),
-                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c]) * scale),
-                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 1]) * scale),
-                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 2]) * scale),
-                     __float_as_uint(__uint_as_float(v[rr * 32 + 4 * c + 3]) * scale));
+        st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * c]) * scale),
+                     __float_as_uint(__uint_as_float(v[4 * c + 1]) * scale),
+                     __float_as_uint(__uint_as_float(v[4 * c + 2]) * scale),
+                     __float_as_uint(__uint_as_float(v[4 * c + 3]) * scale));
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -237,13 +238,25 @@ __device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, c
   }
 }
 
-// Drain one fp32 accumulator as bf16 rows (no scale), 64 columns per round.
+// Drain one fp32 accumulator as bf16 rows (no scale), 64 columns per round; with
+// d_next, also rowsum(value o val) of the written (bf16) values, one float per row.
 template <int D>
 __device__ __forceinline__ void epi_acc_bf16(uint32_t taddr, uint32_t xp, int lane, const EpiRows& R,
-                                             __nv_bfloat16* out) {
+                                             __nv_bfloat16* out, const __nv_bfloat16* val, float* d_next) {
   const int lr = lane >> 3, lc = lane & 7;
+  float dn[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dn[i] = 0.f;
 #pragma unroll 1
   for (int h = 0; h < D / 64; ++h) {
+    uint4 y[8];
+    if (d_next != nullptr) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        y[i] = ((R.live >> (4 * i + lr)) & 1u)
+                   ? __ldg(reinterpret_cast<const uint4*>(val + size_t(R.tok[i]) * D + h * 64 + lc * 8))
+                   : make_uint4(0, 0, 0, 0);
+    }
     uint32_t o[64];
     tmem_ld64(taddr + h * 64, o);
 #pragma unroll
@@ -259,8 +272,19 @@ __device__ __forceinline__ void epi_acc_bf16(uint32_t taddr, uint32_t xp, int la
       const int r = 4 * i + lr;
       const uint4 x = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
       if ((R.live >> r) & 1u) *reinterpret_cast<uint4*>(out + size_t(R.tok[i]) * D + h * 64 + lc * 8) = x;
+      if (d_next != nullptr) dn[i] = dot8_bf16(x, y[i], dn[i]);
     }
     __syncwarp();
+  }
+  if (d_next != nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float v = dn[i];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      if (lc == 0 && ((R.live >> (4 * i + lr)) & 1u)) d_next[R.tok[i]] = v;
+    }
   }
 }
 
@@ -471,14 +495,43 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
       for (int qb = 0; qb < nt; ++qb, ++t) {
         // per-query statistics of the block's query box: row r publishes column r
         float* vl = vec + (t & 1u) * 256;
-        float l = INFINITY, dd = 0.f;  // query columns past the problem: P = 0
-        if (row < tile_valid_rows(g, qb)) {
-          const int tok = base + tile_row_offset(g, qb, row);
-          l = args.lse[tok] * log2e;
-          dd = row_dot<D>(args.dout + size_t(tok) * D, args.out + size_t(tok) * D);
+        const bool qlive = row < tile_valid_rows(g, qb);
+        const int tok = qlive ? base + tile_row_offset(g, qb, row) : 0;
+        vl[row] = qlive ? args.lse[tok] * log2e : INFINITY;  // query columns past the problem: P = 0
+        if (args.Drow != nullptr) {
+          vl[128 + row] = qlive ? args.Drow[tok] : 0.f;
+        } else {
+          // D of the warp's 32 rows: lane l takes rows 4i + l/8, 16-byte chunks l%8 (+8), so
+          // each load instruction reads four whole 128-byte lines; eight lanes sum a row
+          const int lr = lane >> 3, lc = lane & 7;
+          const uint32_t qmask = __ballot_sync(0xffffffffu, qlive);
+#pragma unroll
+          for (int i0 = 0; i0 < 8; i0 += 4) {
+            float part[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int r = 4 * (i0 + u) + lr;
+              const size_t rt = size_t(__shfl_sync(0xffffffffu, tok, r)) * D;
+              part[u] = 0.f;
+              if ((qmask >> r) & 1u) {
+#pragma unroll
+                for (int j = 0; j < D / 64; ++j) {
+                  const uint4 x = __ldg(reinterpret_cast<const uint4*>(args.dout + rt + j * 64 + lc * 8));
+                  const uint4 y = __ldg(reinterpret_cast<const uint4*>(args.out + rt + j * 64 + lc * 8));
+                  part[u] = dot8_bf16(x, y, part[u]);
+                }
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float v = part[u];
+              v += __shfl_xor_sync(0xffffffffu, v, 1);
+              v += __shfl_xor_sync(0xffffffffu, v, 2);
+              v += __shfl_xor_sync(0xffffffffu, v, 4);
+              if (lc == 0) vl[128 + warp * 32 + 4 * (i0 + u) + lr] = v;
+            }
+          }
         }
-        vl[row] = l;
-        vl[128 + row] = dd;
         mbar_arrive(&bars[G_VEC]);
         if (!(ok = wwait(&bars[G_VEC], t & 1u))) break;
         if (!(ok = wwait(&bars[G_SFULL], t & 1u))) break;
@@ -554,7 +607,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
       const EpiRows RK = epi_rows_of(lane, livek ? base + tile_row_offset(g, kb, row) : 0, livek);
       if (!(ok = wwait(&bars[G_ITEMACC], i & 1u))) break;
       tc_fence_after();
-      epi_acc_bf16<D>(tmem + lane_sel + Lay::TM_DV, xp, lane, RK, args.out_val);
+      epi_acc_bf16<D>(tmem + lane_sel + Lay::TM_DV, xp, lane, RK, args.out_val, args.val, args.d_next);
       epi_acc<D, OUT_F32 ? EPI_F32 : EPI_BF16>(tmem + lane_sel + Lay::TM_DK, xp, lane, RK, args.scale, args.add_k,
                                                args.out_k);
       tc_fence_before();

@@ -402,12 +402,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
-    for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
-      const Item it = decode_item(args, i);
-      const PassArgs& P = args.ps[it.pass];
+    // The next job of this warpgroup and this thread's output row in it, found while the
+    // tensor core runs the current job's last P.V (the index arithmetic has divisions).
+    struct SJob {
+      int i;     // item index (>= total_items: none left)
+      int pass;  // 0 local, 1 global
+      int qt;    // query box within the problem
+      int base;  // first token of the problem
+      int tok;   // this thread's output row, or -1 past the box's valid rows
+    };
+    auto find_job = [&](int i) -> SJob {
+      for (; i < args.total_items; i += gridDim.x) {
+        const Item it = decode_item(args, i);
+        const Job J = job_of(args, it, a);
+        if (!J.valid) continue;
+        const Geom& g = args.ps[it.pass].g;
+        const int tok = row < tile_valid_rows(g, J.qt) ? J.base + tile_row_offset(g, J.qt, row) : -1;
+        return SJob{i, it.pass, J.qt, J.base, tok};
+      }
+      return SJob{args.total_items, 0, 0, 0, -1};
+    };
+    SJob cur = find_job(blockIdx.x);
+    while (ok && cur.i < args.total_items) {
+      const PassArgs& P = args.ps[cur.pass];
       const Geom& g = P.g;
-      const Job J = job_of(args, it, a);
-      if (!J.valid) continue;
       float m_run = -INFINITY, l_run = 0.f;
       for (int k = 0; k < g.nt; ++k) {
         if (!(ok = wwait(&bars[F_SF + a], sc & 1))) break;
@@ -471,22 +489,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         m_run = m_use;
       }
       if (!ok) break;
+      const SJob nxt = find_job(cur.i + gridDim.x);
       // ---- epilogue: O / l -> bf16, each thread writes its own output row (16-byte stores)
       pvseen += g.nt;
       if (!(ok = wwait(&bars[F_OF + a], (pvseen - 1) & 1))) break;
       tc_fence_after();
-      const int nvq = tile_valid_rows(g, J.qt);
-      const bool live = row < nvq;
-      const size_t tok = live ? size_t(J.base + tile_row_offset(g, J.qt, row)) : 0;
+      const bool live = cur.tok >= 0;
+      const size_t tok = live ? size_t(cur.tok) : 0;
       {
         // Each thread holds its own row. A warp passes its 32 rows through a private
         // 128B-swizzled patch so that every global store writes four whole 128-byte lines.
         const float inv = 1.f / l_run;
         const uint32_t xp = sbase + Lay::XP_OFF + (warp & 7) * 4096;
         const int lr = lane >> 3, lc = lane & 7;  // read-back: row 4*i + lr, 16-byte chunk lc
+        int rtok[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) rtok[i] = __shfl_sync(0xffffffffu, cur.tok, 4 * i + lr);
         // fused launch: O1 rows are read again by the global pass (keep); O rows are final (drop first)
         const uint64_t pol_out = !fused ? make_policy_evict_normal()
-                                 : it.pass == 0 ? make_policy_evict_last() : make_policy_evict_first();
+                                 : cur.pass == 0 ? make_policy_evict_last() : make_policy_evict_first();
         uint8_t* outb = static_cast<uint8_t*>(P.out);
 #pragma unroll 1
         for (int h = 0; h < D / 64; ++h) {
@@ -503,17 +524,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const int r = 4 * i + lr;  // row of this warp (lane r owns it)
-            const size_t rtok = __shfl_sync(0xffffffffu, tok, r);
-            const bool rlive = __shfl_sync(0xffffffffu, live, r);
             const uint4 val = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
-            if (rlive) st_global_v4_hint(outb + rtok * D * 2 + h * 128 + lc * 16, val, pol_out);
+            if (rtok[i] >= 0) st_global_v4_hint(outb + size_t(rtok[i]) * D * 2 + h * 128 + lc * 16, val, pol_out);
           }
           __syncwarp();
         }
       }
       tc_fence_before();
-      if (fused && it.pass == 0) red_release_cta_shared_add(&rows_done[a], 1u);  // warp 10 publishes
-      if (live && args.discard_base != nullptr && it.pass == 1 && g.nt == 1) {
+      if (fused && cur.pass == 0) red_release_cta_shared_add(&rows_done[a], 1u);  // warp 10 publishes
+      if (live && args.discard_base != nullptr && cur.pass == 1 && g.nt == 1) {
         // this row of the local-pass output was read once, as a value of this group: drop it from L2
         const uint8_t* l1row = args.discard_base + tok * D * 2;
 #pragma unroll
@@ -521,6 +540,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (P.lse != nullptr && live)
         P.lse[tok] = (m_run * c2 + log2f(l_run)) * 0.69314718055994530942f;
+      cur = nxt;
     }
   }
 

@@ -14,6 +14,13 @@ With N > 1 (torchrun, one rank per GPU) every rank runs the full workload on its
 own GPU (independent (batch, head) problems: weak scaling, no data-path
 collective); the timed region is bracketed by barriers and the slowest rank's
 time is reported. Rank 0 prints one JSON line.
+
+Besides the headline the line carries: per-pass kernel times and the roofline of the
+fused launch, an end-to-end number through the public API with host buffers, the
+training step (forward + backward, B=2), the forward of the other timed shapes
+(small_bf16 and long_video, the latter next to dense softmax attention on the same
+Q, K, V as the quadratic teacher, timed through torch's library SDPA) and the fp64
+oracle timed on a bounded sample on the host cores.
 """
 from __future__ import annotations
 
@@ -47,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training-step leg")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the forward timing of the other configs (small_bf16, long_video + dense teacher)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="oracle time budget for the CPU baseline")
     ap.add_argument("--profile-bwd", action="store_true",
                     help="profiling driver for the backward: one warm-up then one forward+backward of the "
@@ -428,6 +437,48 @@ def main():
                  "note": "backward: one fused tcgen05 kernel per pass (dQ parts of multi-box problems added with vector reductions, then one fp32-to-bf16 pass)"}
         del tq, tk, tv, tdo
 
+    # ---------------- the other timed configs: small_bf16, long_video (+ dense softmax teacher)
+    configs = None
+    if not args.no_configs:
+        configs = {}
+
+        def time_flushed(fn, nrep):
+            fn()
+            ts = []
+            for _ in range(nrep):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
+                ts.append((a, b))
+            torch.cuda.synchronize()
+            return sorted(x.elapsed_time(y) for x, y in ts)[nrep // 2]  # median
+
+        for name in ("small_bf16", "long_video"):
+            owl = WORKLOADS[name]
+            oin = make_inputs(owl)
+            oq, okk, ov = (t.to(dev) for t in (oin.q, oin.k, oin.v))
+            del oin
+            oo = torch.empty_like(oq)
+            odesc = sq.make_desc(oq, owl.grid, owl.tile, None)
+            ows = torch.empty(sq.workspace_size(odesc, 0), device=dev, dtype=torch.uint8)
+            oms = time_flushed(lambda: sq.squad_attn_fwd(oq, okk, ov, owl.grid, owl.tile, save=False, out=oo,
+                                                          workspace=ows), 20)
+            sq.poll_device_error()
+            entry = {"ms": oms, "TFLOP/s": owl.fwd_flops() / oms / 1e9, "useful_flops": owl.fwd_flops(),
+                     "n": owl.n, "heads": owl.heads, "grid": list(owl.grid), "tile": list(owl.tile),
+                     "timing": "median of 20 calls, L2 flushed before each"}
+            if name == "long_video":
+                # the quadratic teacher: dense softmax attention on the same Q, K, V (library call)
+                dflops = 4.0 * owl.n * owl.n * owl.d * owl.B * owl.heads
+                dms = time_flushed(lambda: torch.nn.functional.scaled_dot_product_attention(oq, okk, ov), 3)
+                entry["dense_teacher"] = {"ms": dms, "TFLOP/s": dflops / dms / 1e9, "flops": dflops,
+                                          "impl": "torch scaled_dot_product_attention, bf16 (library call)",
+                                          "speedup_of_squad": dms / oms}
+            configs[name] = entry
+            del oq, okk, ov, oo, ows
+
     # ---------------- CPU baseline: the oracle on host cores, rank 0 at N=1 only
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -450,7 +501,7 @@ def main():
                                   "measured_sustained": value / world / peaks.get("bf16_tflops_sustained", 1),
                                   "spec_dense_2250": value / world / 2250.0, "source": peak_src},
             "roofline": roofline, "passes": passes, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks, "train_step": train,
+            "gpu_launches": args.steps, "clocks": clocks, "train_step": train, "configs": configs,
         }
         print(json.dumps(line))
     if world > 1:

@@ -118,6 +118,7 @@ def test_small_bf16_forward(cuda_ok):
     ((2, 44, 40), (1, 22, 20), 2, 128),   # 440-token windows: four boxes, online softmax over two groups
     ((40, 8, 8), (1, 2, 2), 1, 128),      # 640-token groups in the global pass: five boxes, three groups
     ((6, 12, 16), (2, 6, 8), 2, 64),      # tT > 1, d = 64
+    ((2, 44, 40), (1, 22, 20), 1, 64),    # d = 64 with 440-token windows (four boxes)
     ((3, 5, 7), (3, 5, 7), 2, 128),       # one window: the global pass has one token
     ((2, 6, 10), (1, 1, 1), 1, 128),      # one-token windows: the local pass is the identity
     ((9, 6, 6), (3, 2, 3), 3, 128),       # odd sizes everywhere
@@ -165,6 +166,8 @@ def test_long_video_forward_full_size(cuda_ok):
     ((2, 44, 40), (1, 22, 20), 1, 128),   # 440-token windows: four boxes per problem
     ((40, 8, 8), (1, 2, 2), 1, 128),      # 640-token global groups: five boxes
     ((6, 12, 16), (2, 6, 8), 2, 64),      # tT > 1, d = 64
+    ((2, 44, 40), (1, 22, 20), 1, 64),    # d = 64, four key boxes: dQ parts added with reductions
+    ((40, 8, 8), (1, 2, 2), 1, 64),       # d = 64, 640-token global groups: fp32 dQ parts
     ((3, 5, 7), (3, 5, 7), 1, 128),       # one window
     ((2, 6, 10), (1, 1, 1), 1, 128),      # one-token windows
 ])
@@ -172,6 +175,15 @@ def test_bf16_backward_shapes(cuda_ok, grid, tile, heads, d):
     inp = random_problem(23, 1, heads, d, grid, tile, dtype=torch.bfloat16, with_do=True)
     got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
     ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
+        assert_close(a, b, GRAD_MAX, name)
+
+
+def test_bf16_backward_batch_and_explicit_scale(cuda_ok):
+    grid, tile = (4, 22, 40), (1, 11, 20)
+    inp = random_problem(41, 2, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    got = gpu_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile, scale=0.05)
+    ref = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile, scale=0.05)
     for name, a, b in zip(("dQ", "dK", "dV"), got, ref):
         assert_close(a, b, GRAD_MAX, name)
 

@@ -130,7 +130,12 @@ squad_status squad_attn_fwd_noalloc(const squad_desc* desc, const void* q, const
 /* Backward of the forward for the loss sum(o * dout): writes dq, dk, dv.
  * o, o1, lse1, lse2 are the forward's outputs for the same q, k, v (all
  * required). The global pass is differentiated first (values o1), then the
- * local pass (values v); dq and dk sum both passes' contributions. */
+ * local pass (values v); dq and dk sum both passes' contributions.
+ * bf16: when a window or group spans several 128-row boxes, the parts of dq
+ * from its key boxes are added in fp32 with atomic reductions in whatever
+ * order the hardware runs them, so dq may differ between runs in the last
+ * fp32 bits before its final bf16 rounding; dk, dv and the forward are
+ * bitwise reproducible. */
 squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k, const void* v,
                             const void* o, const void* o1, const float* lse1, const float* lse2,
                             const void* dout, void* dq, void* dk, void* dv, void* workspace,

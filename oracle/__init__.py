@@ -10,7 +10,11 @@ torch's SDPA when one window covers the grid or every window is one token,
 the same two passes written as block-masked dense attention in numpy,
 constant-value rows, permutation equivariance, key-shift invariance, the
 closed-form multiply-add count 2*n*d*(w+m), a hand-derived two-token case
-(tests/golden/), and central finite differences for the backward.
+(tests/golden/), and central finite differences for the backward. The
+k-pass functions (passes over nested tiles) are pinned by their reductions
+to the two-pass oracle and to dense attention when tiles are trivial, by
+three block-masked dense attentions composed in numpy, by their closed-form
+multiply-add count, and by finite differences.
 """
 from __future__ import annotations
 
@@ -53,6 +57,13 @@ def _load():
         lib.oracle_fwd.restype = ctypes.c_int
         lib.oracle_bwd.argtypes = [ctypes.POINTER(_Desc), dp, dp, dp, dp, dp, dp, dp, ctypes.c_int]
         lib.oracle_bwd.restype = ctypes.c_int
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_fwd_multi.argtypes = [ctypes.POINTER(_Desc), ctypes.c_int, ip, dp, dp, dp, dp, dp, dp,
+                                         ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
+        lib.oracle_fwd_multi.restype = ctypes.c_int
+        lib.oracle_bwd_multi.argtypes = [ctypes.POINTER(_Desc), ctypes.c_int, ip, dp, dp, dp, dp, dp, dp, dp,
+                                         ctypes.c_int]
+        lib.oracle_bwd_multi.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -113,4 +124,46 @@ def squad_bwd(q, k, v, dout, grid, tile, scale: Optional[float] = None, threads:
                         _ptr(dq), _ptr(dk), _ptr(dv), int(threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_bwd failed with code {rc}")
+    return dq, dk, dv
+
+
+def _tiles(tiles):
+    flat = [int(x) for t in tiles for x in t]
+    if not tiles or any(len(t) != 3 for t in tiles):
+        raise ValueError("tiles: a non-empty list of (tT, tH, tW)")
+    return len(tiles), (ctypes.c_int * len(flat))(*flat)
+
+
+def squad_fwd_multi(q, k, v, grid, tiles, scale: Optional[float] = None, threads: Optional[int] = None):
+    """Forward of k = len(tiles) + 1 passes over nested tiles (innermost first), fp64.
+
+    Returns (o, inter, lse, macs): inter is [k-1, B,h,n,d] (outputs of passes
+    1..k-1), lse is [k, B,h,n], macs the multiply-adds performed.
+    """
+    lib = _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    desc = _desc(q.shape, grid, tiles[0], scale)
+    nt, tarr = _tiles(tiles)
+    o = np.empty_like(q)
+    inter = np.empty((nt,) + q.shape)
+    lse = np.empty((nt + 1,) + q.shape[:3])
+    macs = ctypes.c_ulonglong(0)
+    rc = lib.oracle_fwd_multi(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(inter),
+                              _ptr(lse), int(threads or default_threads()), ctypes.byref(macs))
+    if rc != 0:
+        raise ValueError(f"oracle_fwd_multi failed with code {rc}")
+    return o, inter, lse, int(macs.value)
+
+
+def squad_bwd_multi(q, k, v, dout, grid, tiles, scale: Optional[float] = None, threads: Optional[int] = None):
+    """Gradients (dq, dk, dv) of sum(O * dout) through the k passes, fp64."""
+    lib = _load()
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    desc = _desc(q.shape, grid, tiles[0], scale)
+    nt, tarr = _tiles(tiles)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = lib.oracle_bwd_multi(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(dout),
+                              _ptr(dq), _ptr(dk), _ptr(dv), int(threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_bwd_multi failed with code {rc}")
     return dq, dk, dv

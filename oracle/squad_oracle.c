@@ -299,3 +299,145 @@ done:
     free(o); free(o1); free(do1); free(l1); free(l2); free(win); free(grp);
     return rc;
 }
+
+/* ---- more than two passes ----
+ *
+ * The pages leave "composing more than two passes" as an outlook (gist.science
+ * technical summary, Significance and Claims). Reading used here: nested tiles
+ * t_1 | t_2 | ... | t_{k-1} | grid (each divides the next along every axis), with
+ * t_0 = 1x1x1 and t_k = the grid. Pass j (1..k) attends among the tokens that lie
+ * in the same t_j-window AND at the same position inside their t_{j-1}-window; the
+ * values of pass j are the output of pass j-1 (V for j = 1), Q and K are the
+ * inputs throughout, and the output is that of pass k. With k = 2 this is the
+ * local pass followed by the global pass above. */
+
+typedef struct {
+    long T, H, W;
+    long in[3], out[3]; /* (t, y, x) extents of the inner and the outer tile */
+} pass_geom;
+
+/* Group key: (outer window, position inside the inner window). */
+static long pass_key(const pass_geom* g, long p) {
+    long x = p % g->W, y = (p / g->W) % g->H, t = p / (g->W * g->H);
+    long win = ((t / g->out[0]) * (g->H / g->out[1]) + y / g->out[1]) * (g->W / g->out[2]) + x / g->out[2];
+    long pos = ((t % g->in[0]) * g->in[1] + y % g->in[1]) * g->in[2] + x % g->in[2];
+    return win * (g->in[0] * g->in[1] * g->in[2]) + pos;
+}
+
+static long* bucket_pass(const pass_geom* g, long n, long nkeys, long L) {
+    long* members = (long*)malloc(sizeof(long) * n);
+    long* fill = (long*)calloc((size_t)nkeys, sizeof(long));
+    if (!members || !fill) { free(members); free(fill); return NULL; }
+    for (long p = 0; p < n; p++) {
+        long kk = pass_key(g, p);
+        members[kk * L + fill[kk]++] = p;
+    }
+    free(fill);
+    return members;
+}
+
+/* Geometry of pass j (1-based) of the k = ntiles + 1 passes; 0 if the tiles do not nest. */
+static int pass_of(const oracle_desc* s, int ntiles, const int* tiles, int j, pass_geom* g) {
+    g->T = s->T; g->H = s->H; g->W = s->W;
+    for (int a = 0; a < 3; a++) {
+        g->in[a] = j == 1 ? 1 : tiles[3 * (j - 2) + a];
+        g->out[a] = j == ntiles + 1 ? (a == 0 ? s->T : a == 1 ? s->H : s->W) : tiles[3 * (j - 1) + a];
+        if (g->in[a] <= 0 || g->out[a] <= 0 || g->out[a] % g->in[a]) return 0;
+    }
+    return s->T % g->out[0] == 0 && s->H % g->out[1] == 0 && s->W % g->out[2] == 0;
+}
+
+static int check_multi(const oracle_desc* s, int ntiles, const int* tiles) {
+    if (s->B <= 0 || s->heads <= 0 || s->d <= 0 || s->T <= 0 || s->H <= 0 || s->W <= 0) return ORACLE_BAD_SHAPE;
+    if (ntiles < 1 || tiles == NULL) return ORACLE_BAD_SHAPE;
+    pass_geom g;
+    for (int j = 1; j <= ntiles + 1; j++)
+        if (!pass_of(s, ntiles, tiles, j, &g)) return ORACLE_BAD_SHAPE;
+    return ORACLE_OK;
+}
+
+/* Forward of the k = ntiles + 1 passes. tiles: 3*ntiles ints (tT, tH, tW), innermost
+ * first. Writes o and, when non-NULL, inter (ntiles consecutive [B, heads, n, d]
+ * tensors: the outputs of passes 1..k-1) and lse (k consecutive [B, heads, n]).
+ * *macs (optional) counts the multiply-adds of scores and value sums. */
+int oracle_fwd_multi(const oracle_desc* s, int ntiles, const int* tiles, const double* q, const double* k,
+                     const double* v, double* o, double* inter, double* lse, int nthreads,
+                     unsigned long long* macs) {
+    int rc = check_multi(s, ntiles, tiles);
+    if (rc) return rc;
+    long n = (long)s->T * s->H * s->W;
+    long nbh = (long)s->B * s->heads;
+    size_t big = (size_t)nbh * n * s->d, small = (size_t)nbh * n;
+    double* ib = inter ? inter : (double*)malloc(sizeof(double) * big * ntiles);
+    double* lb = lse ? lse : (double*)malloc(sizeof(double) * small * (ntiles + 1));
+    if (macs) *macs = 0;
+    if (!ib || !lb) { rc = ORACLE_NO_MEMORY; goto done; }
+    const double* val = v;
+    for (int j = 1; j <= ntiles + 1 && rc == ORACLE_OK; j++) {
+        pass_geom g;
+        pass_of(s, ntiles, tiles, j, &g);
+        long L = (g.out[0] / g.in[0]) * (g.out[1] / g.in[1]) * (g.out[2] / g.in[2]);
+        long* members = bucket_pass(&g, n, n / L, L);
+        if (!members) { rc = ORACLE_NO_MEMORY; break; }
+        job_t jb;
+        memset(&jb, 0, sizeof jb);
+        jb.s = s; jb.n = n; jb.bwd = 0;
+        jb.L = L; jb.nprob = n / L; jb.members = members;
+        jb.q = q; jb.k = k; jb.val = val;
+        jb.out = j == ntiles + 1 ? o : ib + big * (j - 1);
+        jb.lse_out = lb + small * (j - 1);
+        rc = run_pass(&jb, nthreads, macs);
+        free(members);
+        val = jb.out;
+    }
+done:
+    if (!inter) free(ib);
+    if (!lse) free(lb);
+    return rc;
+}
+
+/* Backward of oracle_fwd_multi for the loss sum(O * dout): writes dq, dk, dv. The
+ * forward is recomputed; the passes are differentiated from the last to the first,
+ * each one's value gradient being the upstream gradient of the pass before. */
+int oracle_bwd_multi(const oracle_desc* s, int ntiles, const int* tiles, const double* q, const double* k,
+                     const double* v, const double* dout, double* dq, double* dk, double* dv, int nthreads) {
+    int rc = check_multi(s, ntiles, tiles);
+    if (rc) return rc;
+    long n = (long)s->T * s->H * s->W;
+    long nbh = (long)s->B * s->heads;
+    size_t big = (size_t)nbh * n * s->d, small = (size_t)nbh * n;
+    double* o = (double*)malloc(sizeof(double) * big);
+    double* inter = (double*)malloc(sizeof(double) * big * ntiles);
+    double* lse = (double*)malloc(sizeof(double) * small * (ntiles + 1));
+    double* g_up = (double*)malloc(sizeof(double) * big);   /* upstream gradient of the current pass */
+    double* g_val = (double*)malloc(sizeof(double) * big);  /* gradient of its values */
+    if (!o || !inter || !lse || !g_up || !g_val) { rc = ORACLE_NO_MEMORY; goto done; }
+    rc = oracle_fwd_multi(s, ntiles, tiles, q, k, v, o, inter, lse, nthreads, NULL);
+    if (rc) goto done;
+    memset(dq, 0, sizeof(double) * big);
+    memset(dk, 0, sizeof(double) * big);
+    memcpy(g_up, dout, sizeof(double) * big);
+    for (int j = ntiles + 1; j >= 1 && rc == ORACLE_OK; j--) {
+        pass_geom g;
+        pass_of(s, ntiles, tiles, j, &g);
+        long L = (g.out[0] / g.in[0]) * (g.out[1] / g.in[1]) * (g.out[2] / g.in[2]);
+        long* members = bucket_pass(&g, n, n / L, L);
+        if (!members) { rc = ORACLE_NO_MEMORY; break; }
+        double* dval = j == 1 ? dv : g_val;
+        memset(dval, 0, sizeof(double) * big);
+        job_t jb;
+        memset(&jb, 0, sizeof jb);
+        jb.s = s; jb.n = n; jb.bwd = 1;
+        jb.L = L; jb.nprob = n / L; jb.members = members;
+        jb.q = q; jb.k = k;
+        jb.val = j == 1 ? v : inter + big * (j - 2);
+        jb.dout = g_up; jb.lse_in = lse + small * (j - 1);
+        jb.dq = dq; jb.dk = dk; jb.dval = dval;
+        rc = run_pass(&jb, nthreads, NULL);
+        free(members);
+        if (j > 1) { double* tmp = g_up; g_up = g_val; g_val = tmp; }
+    }
+done:
+    free(o); free(inter); free(lse); free(g_up); free(g_val);
+    return rc;
+}

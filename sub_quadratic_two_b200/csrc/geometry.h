@@ -13,6 +13,12 @@
 //                strides (1, W, H*W); problems indexed by the window.
 //   global pass: box = (window column, window row, window frame),
 //                strides (tW, tH*W, tT*H*W); problems indexed by the position.
+// Composing more than two passes (an outlook of the pages: gist.science technical
+// summary, Significance and Claims) uses nested tiles t_0 = 1 x 1 x 1 | t_1 | ... | t_k = grid:
+// pass j attends among the tokens that share a t_j-window and the position
+// inside their t_{j-1}-window, i.e. a box of (t_j / t_{j-1}) sub-windows at
+// strides t_{j-1}; problems are indexed by (position in t_{j-1}, t_j-window),
+// six digits. The two passes above are j = 1 and j = 2 of k = 2.
 // The tensor-core kernels move a problem through TMA boxes ("tiles") of at most
 // 128 rows; a tile is a sub-box that is cut along b or along c.
 #pragma once
@@ -28,8 +34,10 @@ namespace sq {
 struct Geom {
   int a_n, b_n, c_n;  // problem box extents
   int sA, sB, sC;     // token strides of the box dimensions
-  int p0, p1, p2;     // problem index extents (p0 fastest)
-  int o0, o1, o2;     // token offsets of the problem index dimensions
+  int p0, p1, p2;     // problem index extents (p0 fastest): position in the inner window
+  int o0, o1, o2;     // token offsets of those index dimensions
+  int p3, p4, p5;     // then the outer window (1 when the pass has a single one)
+  int o3, o4, o5;
   int probs;          // problems per (batch, head)
   int L;              // rows per problem
   int n;              // tokens per (batch, head)
@@ -44,8 +52,11 @@ struct Geom {
 // Global token index (b,h offset included) of row 0 of problem `prob`.
 SQ_HD int problem_base(const Geom& g, int prob) {
   const int bh = prob / g.probs, idx = prob - bh * g.probs;
-  const int i0 = idx % g.p0, i1 = (idx / g.p0) % g.p1, i2 = idx / (g.p0 * g.p1);
-  return bh * g.n + i0 * g.o0 + i1 * g.o1 + i2 * g.o2;
+  const int q0 = g.p0 * g.p1 * g.p2;  // problems per outer window
+  const int in = idx % q0, out = idx / q0;
+  const int i0 = in % g.p0, i1 = (in / g.p0) % g.p1, i2 = in / (g.p0 * g.p1);
+  const int i3 = out % g.p3, i4 = (out / g.p3) % g.p4, i5 = out / (g.p3 * g.p4);
+  return bh * g.n + i0 * g.o0 + i1 * g.o1 + i2 * g.o2 + i3 * g.o3 + i4 * g.o4 + i5 * g.o5;
 }
 
 // Token offset of row i (0 <= i < L) of a problem, rows ordered (c, b, a).
@@ -101,25 +112,28 @@ inline bool plan_tiles(Geom& g, int max_rows = 128) {
   return true;
 }
 
-// stage 1 = local (window) pass, stage 2 = global (cross-window) pass.
-inline Geom make_geom(int stage, int B, int heads, int T, int H, int W, int tT, int tH, int tW) {
+// One pass over nested tiles: attention among the tokens that share a
+// (cT, cH, cW)-window and the position inside their (iT, iH, iW)-window. The
+// inner tile divides the outer one and the outer one divides the grid.
+inline Geom make_geom_pass(int B, int heads, int T, int H, int W, int iT, int iH, int iW, int cT, int cH, int cW) {
   Geom g{};
   g.n = T * H * W;
   g.bh = B * heads;
-  if (stage == 1) {
-    g.a_n = tW; g.b_n = tH; g.c_n = tT;
-    g.sA = 1; g.sB = W; g.sC = H * W;
-    g.p0 = W / tW; g.p1 = H / tH; g.p2 = T / tT;
-    g.o0 = tW; g.o1 = tH * W; g.o2 = tT * H * W;
-  } else {
-    g.a_n = W / tW; g.b_n = H / tH; g.c_n = T / tT;
-    g.sA = tW; g.sB = tH * W; g.sC = tT * H * W;
-    g.p0 = tW; g.p1 = tH; g.p2 = tT;
-    g.o0 = 1; g.o1 = W; g.o2 = H * W;
-  }
-  g.probs = g.p0 * g.p1 * g.p2;
+  g.a_n = cW / iW; g.b_n = cH / iH; g.c_n = cT / iT;
+  g.sA = iW; g.sB = iH * W; g.sC = iT * H * W;
+  g.p0 = iW; g.p1 = iH; g.p2 = iT;
+  g.o0 = 1; g.o1 = W; g.o2 = H * W;
+  g.p3 = W / cW; g.p4 = H / cH; g.p5 = T / cT;
+  g.o3 = cW; g.o4 = cH * W; g.o5 = cT * H * W;
+  g.probs = g.p0 * g.p1 * g.p2 * g.p3 * g.p4 * g.p5;
   g.L = g.a_n * g.b_n * g.c_n;
   return g;
+}
+
+// stage 1 = local (window) pass, stage 2 = global (cross-window) pass.
+inline Geom make_geom(int stage, int B, int heads, int T, int H, int W, int tT, int tH, int tW) {
+  return stage == 1 ? make_geom_pass(B, heads, T, H, W, 1, 1, 1, tT, tH, tW)
+                    : make_geom_pass(B, heads, T, H, W, tT, tH, tW, T, H, W);
 }
 
 }  // namespace sq

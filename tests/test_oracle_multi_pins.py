@@ -1,0 +1,151 @@
+"""Pins for the oracle's k-pass functions (passes over nested tiles).
+
+The pages name composing more than two passes as an outlook ("SQuad: Sub-Quadratic
+Attention Distillation for Efficient Video Generation", gist.science technical
+summary, Significance and Claims). Reading: nested tiles t_1 | ... | t_{k-1} | grid;
+pass j attends among tokens in the same t_j-window at the same position inside
+their t_{j-1}-window (t_0 = one token, t_k = the grid), values = previous output.
+Each check below comes from outside the k-pass code: the two-pass oracle (pinned on
+its own), dense attention from torch's SDPA, dense attention with boolean masks
+built from coordinates in numpy, a closed-form multiply-add count, and finite
+differences.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from workloads import random_problem
+
+
+def _coords(grid):
+    T, H, W = grid
+    return np.unravel_index(np.arange(T * H * W), (T, H, W))  # x fastest
+
+
+def _pass_masks(grid, tiles):
+    """Boolean [n, n] masks of every pass, from token coordinates."""
+    c = np.stack(_coords(grid), 1)
+    chain = [(1, 1, 1)] + [tuple(t) for t in tiles] + [tuple(grid)]
+    masks = []
+    for inner, outer in zip(chain[:-1], chain[1:]):
+        win = c // np.array(outer)
+        pos = c % np.array(inner)
+        same = (win[:, None, :] == win[None, :, :]).all(-1) & (pos[:, None, :] == pos[None, :, :]).all(-1)
+        masks.append(torch.from_numpy(same))
+    return masks
+
+
+def _masked_dense_passes(q, k, v, grid, tiles):
+    val = v
+    for m in _pass_masks(grid, tiles):
+        val = F.scaled_dot_product_attention(q, k, val, attn_mask=m)
+    return val
+
+
+def _problem(seed, grid, d=16, heads=2, B=1):
+    inp = random_problem(seed, B, heads, d, grid, (1, 1, 1), dtype=torch.float64, with_do=True)
+    return inp.q, inp.k, inp.v, inp.do
+
+
+def test_one_tile_is_the_two_pass_operator():
+    grid, tile = (2, 4, 6), (1, 2, 3)
+    q, k, v, do = _problem(1, grid)
+    o, inter, lse, _ = oracle.squad_fwd_multi(q, k, v, grid, [tile])
+    ro, ro1, rl1, rl2, _ = oracle.squad_fwd(q, k, v, grid, tile)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(inter[0], ro1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[0], rl1, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse[1], rl2, rtol=0, atol=1e-13)
+    g = oracle.squad_bwd_multi(q, k, v, do, grid, [tile])
+    r = oracle.squad_bwd(q, k, v, do, grid, tile)
+    for a, b in zip(g, r):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_trivial_inner_tile_reduces_to_two_passes():
+    # t_1 = one token: pass 1 is the identity (O1 = V), passes 2 and 3 are SQuad with t_2
+    grid, tile = (2, 4, 8), (2, 2, 4)
+    q, k, v, _ = _problem(2, grid)
+    o, inter, _, _ = oracle.squad_fwd_multi(q, k, v, grid, [(1, 1, 1), tile])
+    ro, _, _, _, _ = oracle.squad_fwd(q, k, v, grid, tile)
+    np.testing.assert_allclose(inter[0], v.numpy(), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+
+
+def test_outer_tile_equal_to_grid_reduces_to_two_passes():
+    # t_2 = grid: the last pass groups single tokens (identity)
+    grid, tile = (2, 4, 8), (1, 2, 4)
+    q, k, v, _ = _problem(3, grid)
+    o, inter, _, _ = oracle.squad_fwd_multi(q, k, v, grid, [tile, grid])
+    ro, _, _, _, _ = oracle.squad_fwd(q, k, v, grid, tile)
+    np.testing.assert_allclose(o, ro, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o, inter[1], rtol=0, atol=1e-15)
+
+
+def test_trivial_tiles_give_dense_attention():
+    grid = (2, 3, 4)
+    q, k, v, _ = _problem(4, grid)
+    o, _, _, _ = oracle.squad_fwd_multi(q, k, v, grid, [(1, 1, 1), (1, 1, 1)])
+    ref = F.scaled_dot_product_attention(q, k, v)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("grid,tiles", [
+    ((2, 4, 8), [(1, 2, 2), (2, 2, 4)]),
+    ((4, 4, 4), [(1, 1, 2), (2, 2, 2)]),
+    ((3, 6, 4), [(1, 3, 1), (3, 3, 2)]),
+    ((2, 4, 8), [(1, 1, 2), (1, 2, 2), (2, 2, 4)]),  # four passes
+])
+def test_passes_equal_masked_dense_attention(grid, tiles):
+    q, k, v, _ = _problem(5, grid)
+    o, _, _, _ = oracle.squad_fwd_multi(q, k, v, grid, tiles)
+    ref = _masked_dense_passes(q, k, v, grid, tiles)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_mac_count_closed_form():
+    # 2 n d sum_j |t_j| / |t_{j-1}| per (batch, head): scores plus value sums
+    grid, tiles = (2, 4, 8), [(1, 2, 2), (2, 2, 4)]
+    q, k, v, _ = _problem(6, grid, d=8, heads=3, B=2)
+    _, _, _, macs = oracle.squad_fwd_multi(q, k, v, grid, tiles)
+    n = 64
+    sizes = [1, 4, 16, n]
+    expect = 2 * 3 * 2 * n * 8 * sum(b // a for a, b in zip(sizes[:-1], sizes[1:]))
+    assert macs == expect
+
+
+def test_backward_matches_autograd_of_masked_dense():
+    grid, tiles = (2, 4, 4), [(1, 2, 1), (2, 2, 2)]
+    q, k, v, do = _problem(7, grid, d=8)
+    qq, kk, vv = (t.clone().requires_grad_(True) for t in (q, k, v))
+    (_masked_dense_passes(qq, kk, vv, grid, tiles) * do).sum().backward()
+    g = oracle.squad_bwd_multi(q, k, v, do, grid, tiles)
+    for a, b in zip(g, (qq.grad, kk.grad, vv.grad)):
+        np.testing.assert_allclose(a, b.numpy(), rtol=0, atol=1e-11)
+
+
+def test_backward_finite_differences():
+    grid, tiles = (2, 2, 4), [(1, 1, 2), (2, 1, 2)]
+    q, k, v, do = _problem(8, grid, d=4, heads=1)
+    dq, dk, dv = oracle.squad_bwd_multi(q, k, v, do, grid, tiles)
+    loss = lambda q_, k_, v_: float((oracle.squad_fwd_multi(q_, k_, v_, grid, tiles)[0] * do.numpy()).sum())
+    eps = 1e-6
+    rng = np.random.default_rng(0)
+    for grad, which in ((dq, 0), (dk, 1), (dv, 2)):
+        for _ in range(4):
+            idx = tuple(int(rng.integers(0, s)) for s in q.shape)
+            args = [q.clone(), k.clone(), v.clone()]
+            args[which][idx] += eps
+            up = loss(*args)
+            args[which][idx] -= 2 * eps
+            dn = loss(*args)
+            assert abs((up - dn) / (2 * eps) - grad[idx]) < 1e-6
+
+
+def test_tiles_that_do_not_nest_are_rejected():
+    q, k, v, _ = _problem(9, (2, 4, 8))
+    for tiles in ([(1, 3, 1)], [(1, 2, 4), (1, 4, 2)], [(2, 2, 2), (1, 1, 1)]):
+        with pytest.raises(ValueError):
+            oracle.squad_fwd_multi(q, k, v, (2, 4, 8), tiles)

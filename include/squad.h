@@ -141,6 +141,47 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
                             const void* dout, void* dq, void* dk, void* dv, void* workspace,
                             size_t workspace_bytes, void* stream);
 
+/* ---- More than two passes ----
+ * The pages name composing more than two passes as an outlook ("SQuad:
+ * Sub-Quadratic Attention Distillation for Efficient Video Generation",
+ * gist.science technical summary, Significance and Claims). Reading: k =
+ * ntiles + 1 passes over nested tiles t_1 | t_2 | ... | t_{k-1} | grid, given
+ * as tiles[3*ntiles] = (tT, tH, tW) innermost first, each dividing the next
+ * (and the last the grid) along every axis; desc->tT, tH, tW are ignored and
+ * 1 <= ntiles <= 4. Pass j attends among the tokens that share a t_j-window and
+ * the position inside their t_{j-1}-window (t_0 = one token, t_k = the grid);
+ * its values are the output of pass j-1 (v for j = 1); q, k and the scale are
+ * those of every pass; the result is the output of pass k. ntiles = 1 is
+ * squad_attn_fwd with tile t_1. Cost: 4 n d (|t_1| + |t_2|/|t_1| + ... +
+ * n/|t_{k-1}|) FLOPs per (batch, head). Each pass is one launch of the
+ * kernels above (no fused hand-off between passes). On bf16 every pass's box
+ * row (t_j / t_{j-1} along W) must be at most 128 tokens (else
+ * SQUAD_ERR_UNSUPPORTED); tiles that do not nest give SQUAD_ERR_SHAPE. */
+
+/* Forward. inter: ntiles consecutive [B, heads, n, d] tensors of the input
+ * dtype receiving the outputs of passes 1..k-1 (required: each is the next
+ * pass's values, and the backward reads them). lse: k consecutive [B, heads, n]
+ * fp32 (natural log), or NULL. o, inter, lse are written, nothing else. */
+squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
+                                  const void* k, const void* v, void* o, void* inter, float* lse, void* stream);
+
+/* Bytes of workspace squad_attn_multi_bwd needs: two upstream-gradient
+ * tensors of the input dtype, four fp32 [B, heads, n, d] accumulators and one
+ * fp32 row vector (each part 256-byte aligned). */
+squad_status squad_attn_multi_bwd_workspace_size(const squad_desc* desc, int ntiles, const int* tiles,
+                                                 size_t* bytes);
+
+/* Backward for the loss sum(o * dout): writes dq, dk, dv. o, inter and lse
+ * (all required) are squad_attn_multi_fwd's outputs for the same inputs. The
+ * passes are differentiated from the last to the first; dq and dk sum every
+ * pass's contribution (in fp32 until the last step). The bf16 dq is
+ * reproducible only up to the fp32 reduction order when a problem spans
+ * several boxes (as for squad_attn_bwd). */
+squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
+                                  const void* k, const void* v, const void* o, const void* inter, const float* lse,
+                                  const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Geometry the kernels use for one pass (stage 1 = local/window pass,
  * stage 2 = global/cross-window pass), for tests and byte accounting.
  * Writes 8 ints to info: [0] rows per problem (w or m), [1] problems per

@@ -5,7 +5,8 @@ Attention Distillation for Efficient Video Generation" (gist.science technical
 summary, Methodology section 1): softmax attention inside each tT x tH x tW
 window of a T x H x W token grid, then softmax attention across windows among
 tokens with the same in-window position, with the first pass's output as
-values. All arithmetic runs in the CUDA kernels of libsquad.so; this module
+values (attention_multi composes more passes over nested tiles). All
+arithmetic runs in the CUDA kernels of libsquad.so; this module
 only checks and marshals arguments (PyTorch supplies device memory and
 streams). There is no CPU fallback: without the built library every call
 raises.
@@ -21,7 +22,7 @@ import torch
 __all__ = [
     "SquadError", "attention", "squad_attn_fwd", "squad_attn_bwd", "workspace_size",
     "poll_device_error", "library_path", "load_library", "SQUAD_F32", "SQUAD_BF16", "squad_attn_fwd_pass",
-    "plan_info", "make_desc",
+    "plan_info", "make_desc", "attention_multi", "squad_attn_multi_fwd", "squad_attn_multi_bwd",
 ]
 
 SQUAD_F32 = 0
@@ -68,11 +69,17 @@ def load_library():
         lib.squad_attn_bwd.argtypes = [dp, vp, vp, vp, vp, vp, fp, fp, vp, vp, vp, vp, vp, sz, vp]
         lib.squad_attn_fwd_pass.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, fp, vp]
         lib.squad_plan_info.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.squad_attn_multi_fwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp]
+        lib.squad_attn_multi_bwd_workspace_size.argtypes = [dp, ctypes.c_int, ip, ctypes.POINTER(ctypes.c_size_t)]
+        lib.squad_attn_multi_bwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp,
+                                             sz, vp]
         lib.squad_poll_device_error.argtypes = [vp]
         lib.squad_strerror.argtypes = [ctypes.c_int]
         lib.squad_strerror.restype = ctypes.c_char_p
         for f in ("squad_attn_workspace_size", "squad_attn_fwd", "squad_attn_bwd", "squad_poll_device_error",
-                  "squad_attn_fwd_pass", "squad_plan_info",
+                  "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_multi_fwd",
+                  "squad_attn_multi_bwd_workspace_size", "squad_attn_multi_bwd",
                   "squad_last_cuda_error", "squad_version"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
@@ -266,3 +273,82 @@ def squad_attn_fwd_noalloc(q, k, v, grid, tile, scale: Optional[float] = None, o
         _check(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse1), _ptr(lse2), st),
                "squad_attn_fwd_noalloc")
     return o
+
+
+# ---------------------------------------------------------------- more than two passes
+
+def _tiles_arg(tiles: Sequence[Sequence[int]]):
+    flat = [int(x) for t in tiles for x in t]
+    if len(tiles) < 1 or any(len(t) != 3 for t in tiles):
+        raise ValueError("tiles: a non-empty sequence of (tT, tH, tW), innermost first")
+    return len(tiles), (ctypes.c_int * len(flat))(*flat)
+
+
+def squad_attn_multi_fwd(q, k, v, grid, tiles, scale: Optional[float] = None,
+                         stream: Optional[torch.cuda.Stream] = None):
+    """k = len(tiles) + 1 passes over nested tiles (innermost first) through the C ABI.
+
+    Returns (o, inter, lse): inter is [k-1, B, heads, n, d] (outputs of passes
+    1..k-1), lse is [k, B, heads, n] fp32.
+    """
+    lib = load_library()
+    _check_inputs(q, k, v)
+    desc = make_desc(q, grid, tiles[0], scale)
+    nt, tarr = _tiles_arg(tiles)
+    o = torch.empty_like(q)
+    inter = torch.empty((nt,) + tuple(q.shape), device=q.device, dtype=q.dtype)
+    lse = torch.empty((nt + 1,) + tuple(q.shape[:3]), device=q.device, dtype=torch.float32)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                        _ptr(inter), _ptr(lse), st), "squad_attn_multi_fwd")
+    return o, inter, lse
+
+
+def squad_attn_multi_bwd(q, k, v, o, inter, lse, dout, grid, tiles, scale: Optional[float] = None,
+                         stream: Optional[torch.cuda.Stream] = None):
+    """Backward of squad_attn_multi_fwd through the C ABI. Returns (dq, dk, dv)."""
+    lib = load_library()
+    _check_inputs(q, k, v, o, dout)
+    desc = make_desc(q, grid, tiles[0], scale)
+    nt, tarr = _tiles_arg(tiles)
+    ws_bytes = ctypes.c_size_t(0)
+    _check(lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(desc), nt, tarr, ctypes.byref(ws_bytes)),
+           "squad_attn_multi_bwd_workspace_size")
+    ws = torch.empty(int(ws_bytes.value), device=q.device, dtype=torch.uint8)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    with torch.cuda.device(q.device):
+        st = _stream_handle(stream, q.device)
+        _check(lib.squad_attn_multi_bwd(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                        _ptr(inter.contiguous()), _ptr(lse.contiguous()), _ptr(dout), _ptr(dq),
+                                        _ptr(dk), _ptr(dv), _ptr(ws), int(ws_bytes.value), st),
+               "squad_attn_multi_bwd")
+    return dq, dk, dv
+
+
+class _SquadAttentionMulti(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, grid, tiles, scale):
+        o, inter, lse = squad_attn_multi_fwd(q, k, v, grid, tiles, scale)
+        if any(ctx.needs_input_grad[:3]):
+            ctx.save_for_backward(q, k, v, o, inter, lse)
+        ctx.geom = (tuple(grid), tuple(tuple(t) for t in tiles), scale)
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, inter, lse = ctx.saved_tensors
+        grid, tiles, scale = ctx.geom
+        dq, dk, dv = squad_attn_multi_bwd(q, k, v, o, inter, lse, dout.contiguous(), grid, tiles, scale)
+        return dq, dk, dv, None, None, None
+
+
+def attention_multi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tuple[int, int, int],
+                    tiles: Sequence[Tuple[int, int, int]], scale: Optional[float] = None) -> torch.Tensor:
+    """k = len(tiles) + 1 passes over nested tiles (innermost first), differentiable.
+
+    Pass j attends among the tokens of one t_j-window at the same position inside
+    their t_{j-1}-window (t_0 = one token, the last window the whole grid); one
+    tile gives attention(q, k, v, grid, tiles[0]).
+    """
+    return _SquadAttentionMulti.apply(q, k, v, tuple(grid), tuple(tuple(t) for t in tiles), scale)

@@ -98,7 +98,8 @@ struct Plan {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-squad_status make_plan(const squad_desc* d, Plan* p) {
+// with_passes = false checks the tensors only (the k-pass entry points plan their own passes)
+squad_status make_plan(const squad_desc* d, Plan* p, bool with_passes = true) {
   if (d == nullptr) return SQUAD_ERR_INVALID_ARG;
   if (d->dtype != SQUAD_F32 && d->dtype != SQUAD_BF16) return SQUAD_ERR_INVALID_ARG;
   if (d->B <= 0 || d->heads <= 0 || d->d <= 0 || d->T <= 0 || d->H <= 0 || d->W <= 0 || d->tT <= 0 ||
@@ -114,10 +115,12 @@ squad_status make_plan(const squad_desc* d, Plan* p) {
   } else {
     if (d->d % 32 != 0 || d->d > 256) return SQUAD_ERR_UNSUPPORTED;
   }
-  p->g1 = sq::make_geom(1, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
-  p->g2 = sq::make_geom(2, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
-  if (d->dtype == SQUAD_BF16) {
-    if (!sq::plan_tiles(p->g1) || !sq::plan_tiles(p->g2)) return SQUAD_ERR_UNSUPPORTED;
+  if (with_passes) {
+    p->g1 = sq::make_geom(1, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
+    p->g2 = sq::make_geom(2, d->B, d->heads, d->T, d->H, d->W, d->tT, d->tH, d->tW);
+    if (d->dtype == SQUAD_BF16) {
+      if (!sq::plan_tiles(p->g1) || !sq::plan_tiles(p->g2)) return SQUAD_ERR_UNSUPPORTED;
+    }
   }
   p->rows = rows;
   p->elem = d->dtype == SQUAD_BF16 ? 2 : 4;
@@ -668,5 +671,195 @@ const char* squad_strerror(int status) {
 int squad_last_cuda_error(void) { return t_last_cuda; }
 
 int squad_version(void) { return kVersion; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- more than two passes
+// k = ntiles + 1 passes over nested tiles t_1 | ... | t_{k-1} | grid (innermost first):
+// pass j attends among the tokens of one t_j-window at the same position inside their
+// t_{j-1}-window; its values are the previous pass's output. The pages name composing
+// more than two passes as an outlook (gist.science technical summary, Significance and
+// Claims); k = 2 is the operator above. Each pass runs on the same kernels as the two
+// SQuad passes, one launch per pass.
+
+namespace {
+
+constexpr int kMaxTiles = 4;
+
+struct MultiPlan {
+  Plan base;                 // scale, rows, element size (its g1/g2 are unused)
+  int k;                     // passes
+  Geom g[kMaxTiles + 1];     // pass j at g[j - 1]
+};
+
+squad_status make_multi_plan(const squad_desc* d, int ntiles, const int* tiles, MultiPlan* mp) {
+  if (d == nullptr || tiles == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (ntiles < 1 || ntiles > kMaxTiles) return SQUAD_ERR_UNSUPPORTED;
+  // the base plan validates the tensors; the tiles are checked here (nested)
+  squad_desc d1 = *d;
+  d1.tT = d1.tH = d1.tW = 1;
+  squad_status s = make_plan(&d1, &mp->base, false);
+  if (s != SQUAD_OK) return s;
+  mp->k = ntiles + 1;
+  const int grid[3] = {d->T, d->H, d->W};
+  for (int j = 1; j <= mp->k; ++j) {
+    int in[3], out[3];
+    for (int a = 0; a < 3; ++a) {
+      in[a] = j == 1 ? 1 : tiles[3 * (j - 2) + a];
+      out[a] = j == mp->k ? grid[a] : tiles[3 * (j - 1) + a];
+      if (in[a] <= 0 || out[a] <= 0 || out[a] % in[a] != 0 || grid[a] % out[a] != 0) return SQUAD_ERR_SHAPE;
+    }
+    Geom g = sq::make_geom_pass(d->B, d->heads, d->T, d->H, d->W, in[0], in[1], in[2], out[0], out[1], out[2]);
+    if (d->dtype == SQUAD_BF16 && !sq::plan_tiles(g)) return SQUAD_ERR_UNSUPPORTED;
+    mp->g[j - 1] = g;
+  }
+  return SQUAD_OK;
+}
+
+// Backward workspace: two upstream gradients (dtype) used in turn, two fp32 dQ and two
+// fp32 dK accumulators used in turn (the pass reads one and writes the other), one fp32
+// row vector.
+struct MultiWs {
+  size_t up[2], dq[2], dk[2], drow, total;
+};
+
+MultiWs multi_workspace(const MultiPlan& mp, const squad_desc* d) {
+  MultiWs w{};
+  const size_t big = size_t(mp.base.rows) * d->d;
+  size_t off = 0;
+  for (int i = 0; i < 2; ++i) { w.up[i] = off; off += align256(big * mp.base.elem); }
+  for (int i = 0; i < 2; ++i) { w.dq[i] = off; off += align256(big * 4); }
+  for (int i = 0; i < 2; ++i) { w.dk[i] = off; off += align256(big * 4); }
+  w.drow = off;
+  off += align256(size_t(mp.base.rows) * 4);
+  w.total = off;
+  return w;
+}
+
+template <int DPL>
+squad_status simt_pass_bwd_f32(const Geom& g, long long rows, const float* q, const float* k, const float* val,
+                               const float* out, const float* dout, const float* lse, float* Drow,
+                               const float* dq_add, float* dq, const float* dk_add, float* dk, float* dval, int d,
+                               float scale, cudaStream_t st) {
+  return simt_pass_bwd_t<float, float, float, float, DPL>(g, rows, q, k, val, out, dout, lse, Drow, dq_add, dq,
+                                                          dk_add, dk, dval, d, scale, st);
+}
+
+squad_status simt_pass_bwd_f32_any(int d, const Geom& g, long long rows, const float* q, const float* k,
+                                   const float* val, const float* out, const float* dout, const float* lse,
+                                   float* Drow, const float* dq_add, float* dq, const float* dk_add, float* dk,
+                                   float* dval, float scale, cudaStream_t st) {
+  switch (d / 32) {
+#define SQ_CASE(n) \
+  case n: return simt_pass_bwd_f32<n>(g, rows, q, k, val, out, dout, lse, Drow, dq_add, dq, dk_add, dk, dval, d, scale, st);
+    SQ_CASE(1) SQ_CASE(2) SQ_CASE(3) SQ_CASE(4) SQ_CASE(5) SQ_CASE(6) SQ_CASE(7) SQ_CASE(8)
+#undef SQ_CASE
+  }
+  return SQUAD_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+extern "C" {
+
+squad_status squad_attn_multi_bwd_workspace_size(const squad_desc* desc, int ntiles, const int* tiles,
+                                                 size_t* bytes) {
+  MultiPlan mp;
+  squad_status s = make_multi_plan(desc, ntiles, tiles, &mp);
+  if (s != SQUAD_OK) return s;
+  if (bytes == nullptr) return SQUAD_ERR_INVALID_ARG;
+  *bytes = multi_workspace(mp, desc).total;
+  return SQUAD_OK;
+}
+
+squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
+                                  const void* k, const void* v, void* o, void* inter, float* lse, void* stream) {
+  MultiPlan mp;
+  squad_status s = make_multi_plan(desc, ntiles, tiles, &mp);
+  if (s != SQUAD_OK) return s;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(inter)})
+    if (ptr == nullptr) return SQUAD_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(inter),
+                          static_cast<const void*>(lse)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t big = size_t(mp.base.rows) * desc->d * mp.base.elem;
+  const void* val = v;
+  for (int j = 1; j <= mp.k; ++j) {
+    void* out = j == mp.k ? o : static_cast<uint8_t*>(inter) + big * (j - 1);
+    float* l = lse == nullptr ? nullptr : lse + size_t(mp.base.rows) * (j - 1);
+    if (desc->dtype == SQUAD_BF16) {
+      Plan p = mp.base;
+      p.g1 = p.g2 = mp.g[j - 1];
+      s = launch_fwd_tc(ds, desc->d, sq::FWD_LOCAL, p, q, k, val, out, l, val, out, l, nullptr, nullptr, st);
+    } else {
+      s = simt_fwd<float>(mp.g[j - 1], q, k, val, out, l, desc->d, mp.base.scale, st);
+    }
+    if (s != SQUAD_OK) return s;
+    val = out;
+  }
+  return SQUAD_OK;
+}
+
+squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
+                                  const void* k, const void* v, const void* o, const void* inter, const float* lse,
+                                  const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  MultiPlan mp;
+  squad_status s = make_multi_plan(desc, ntiles, tiles, &mp);
+  if (s != SQUAD_OK) return s;
+  for (const void* ptr : {q, k, v, o, inter, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (ptr == nullptr) return SQUAD_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, inter, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv),
+                          static_cast<const void*>(workspace)})
+    if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  const MultiWs w = multi_workspace(mp, desc);
+  if (workspace == nullptr || workspace_bytes < w.total) return SQUAD_ERR_WORKSPACE;
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t big = size_t(mp.base.rows) * desc->d * mp.base.elem;
+  const bool bf16 = desc->dtype == SQUAD_BF16;
+  auto inter_at = [&](int j) -> const void* { return static_cast<const uint8_t*>(inter) + big * (j - 1); };
+  // Last pass first. Pass j reads the upstream gradient of its output and writes that of
+  // its values (the output of pass j-1); dQ and dK accumulate in fp32 across passes (each
+  // pass reads the sum so far from one buffer and writes the new sum to the other), and
+  // the first pass writes the final dq, dk, dv.
+  const void* up = dout;
+  int acc = 0;  // accumulator holding the sum so far (valid for j < k)
+  for (int j = mp.k; j >= 1; --j) {
+    const Geom& g = mp.g[j - 1];
+    const void* val = j == 1 ? v : inter_at(j - 1);
+    const void* out = j == mp.k ? o : inter_at(j);
+    const float* l = lse + size_t(mp.base.rows) * (j - 1);
+    void* dval = j == 1 ? dv : ws + w.up[j & 1];
+    const float* q_add = j == mp.k ? nullptr : reinterpret_cast<const float*>(ws + w.dq[acc]);
+    const float* k_add = j == mp.k ? nullptr : reinterpret_cast<const float*>(ws + w.dk[acc]);
+    void* q_out = j == 1 ? dq : ws + w.dq[acc ^ 1];
+    void* k_out = j == 1 ? dk : ws + w.dk[acc ^ 1];
+    if (bf16) {
+      // the last step (j = 1) writes bf16 and, for multi-box problems, adds its dQ parts
+      // into the fp32 sum before the conversion
+      float* q_acc = j == 1 ? const_cast<float*>(q_add) : nullptr;
+      s = tc_pass_bwd(ds, mp.base, desc->d, g, q, k, val, out, up, l, nullptr, nullptr, q_add, q_acc, q_out,
+                      k_add, k_out, static_cast<__nv_bfloat16*>(dval), j > 1, st);
+    } else {
+      s = simt_pass_bwd_f32_any(desc->d, g, mp.base.rows, static_cast<const float*>(q),
+                                static_cast<const float*>(k), static_cast<const float*>(val),
+                                static_cast<const float*>(out), static_cast<const float*>(up), l,
+                                reinterpret_cast<float*>(ws + w.drow), q_add, static_cast<float*>(q_out), k_add,
+                                static_cast<float*>(k_out), static_cast<float*>(dval), mp.base.scale, st);
+    }
+    if (s != SQUAD_OK) return s;
+    up = dval;
+    acc ^= 1;
+  }
+  return SQUAD_OK;
+}
 
 }  // extern "C"

@@ -135,3 +135,44 @@ def test_plan_tiles_cover_problem(lib):
             L, probs, nt, box, a, b, c, kt = _plan(lib, d, stage)
             assert box == a * b * c <= 128
             assert (nt - 1) * box < L <= nt * box
+
+
+# ---------------------------------------------------------------- more than two passes
+
+def _tiles(*ts):
+    flat = [x for t in ts for x in t]
+    return len(ts), (ctypes.c_int * len(flat))(*flat)
+
+
+def _mfwd(lib, desc, tiles, o=FAKE, inter=FAKE, lse=None):
+    nt, arr = tiles
+    return lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, arr, FAKE, FAKE, FAKE, o, inter, lse, None)
+
+
+def test_multi_pass_argument_errors(lib):
+    d = _desc(T=4, H=8, W=8)
+    assert _mfwd(lib, d, _tiles((1, 2, 2), (1, 3, 4))) == SHAPE          # 2 does not divide 3
+    assert _mfwd(lib, d, _tiles((1, 4, 4), (1, 2, 2))) == SHAPE          # outer tile smaller than inner
+    assert _mfwd(lib, d, _tiles((1, 2, 2), (3, 4, 4))) == SHAPE          # 3 does not divide T=4
+    assert _mfwd(lib, d, _tiles(*[(1, 1, 1)] * 5)) == UNSUPPORTED        # at most four tiles
+    assert lib.squad_attn_multi_fwd(ctypes.byref(d), 1, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == INVALID
+    assert _mfwd(lib, d, _tiles((1, 2, 2), (1, 4, 4)), inter=None) == INVALID
+    assert _mfwd(lib, d, _tiles((1, 2, 2), (1, 4, 4)), o=MISALIGNED) == ALIGN
+    # bf16: a pass whose box row (t_j / t_{j-1} along W) exceeds 128 tokens
+    wide = _desc(T=1, H=1, W=512, tT=1, tH=1, tW=1)
+    assert _mfwd(lib, wide, _tiles((1, 1, 2), (1, 1, 512))) == UNSUPPORTED
+    nt, arr = _tiles((1, 2, 2), (1, 4, 4))
+    need = ctypes.c_size_t(0)
+    assert lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(d), nt, arr, ctypes.byref(need)) == OK
+    args = [FAKE] * 10  # q, k, v, o, inter, lse, dout, dq, dk, dv
+    assert lib.squad_attn_multi_bwd(ctypes.byref(d), nt, arr, *args, FAKE, need.value - 16, None) == WORKSPACE
+
+
+def test_multi_pass_workspace_size(lib):
+    d = _desc(T=4, H=8, W=8)
+    nt, arr = _tiles((1, 2, 2), (1, 4, 4))
+    got = ctypes.c_size_t(0)
+    assert lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(d), nt, arr, ctypes.byref(got)) == OK
+    rows = 1 * 2 * 256
+    # two bf16 upstream gradients, four fp32 accumulators, one fp32 row vector
+    assert got.value == 2 * rows * 128 * 2 + 4 * rows * 128 * 4 + rows * 4

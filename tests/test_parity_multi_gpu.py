@@ -1,0 +1,114 @@
+"""GPU parity of the k-pass entry points (passes over nested tiles) against the oracle.
+
+Same tolerances as the two-pass operator: fp32 max |err| <= 1e-5; bf16 forward
+max <= 1.5e-2 and mean <= 2e-3; bf16 gradients max <= 3e-2. Reading of the
+pages' outlook on composing more than two passes ("SQuad: Sub-Quadratic
+Attention Distillation for Efficient Video Generation", gist.science technical
+summary, Significance and Claims): nested tiles, pass j attends within a
+t_j-window among tokens at the same position in their t_{j-1}-window.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sub_quadratic_two_b200 as sq
+from workloads import WORKLOADS, make_inputs, random_problem
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+BF16_MAX, BF16_MEAN, GRAD_MAX = 1.5e-2, 2e-3, 3e-2
+
+
+def _np(t):
+    return t.detach().cpu().double().numpy()
+
+
+def _err(a, b):
+    e = np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))
+    return float(e.max()), float(e.mean())
+
+
+def _gpu_fwd_bwd(inp, grid, tiles, scale=None):
+    q, k, v, do = (t.contiguous().cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+    o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, grid, tiles, scale)
+    grads = sq.squad_attn_multi_bwd(q, k, v, o, inter, lse, do, grid, tiles, scale)
+    sq.poll_device_error()
+    return o, inter, lse, grads
+
+
+@pytest.mark.parametrize("grid,tiles,d", [
+    ((2, 4, 8), [(1, 2, 2), (2, 2, 4)], 64),
+    ((2, 4, 8), [(1, 1, 2), (1, 2, 2), (2, 2, 4)], 32),   # four passes
+    ((3, 6, 4), [(1, 3, 1), (3, 3, 2)], 96),
+])
+def test_fp32_passes_forward_and_backward(cuda_ok, grid, tiles, d):
+    inp = random_problem(51, 2, 2, d, grid, (1, 1, 1), dtype=torch.float32, with_do=True)
+    o, inter, lse, grads = _gpu_fwd_bwd(inp, grid, tiles)
+    ro, rinter, rlse, _ = oracle.squad_fwd_multi(inp.q, inp.k, inp.v, grid, tiles)
+    assert _err(_np(o), ro)[0] <= F32_TOL
+    assert _err(_np(inter), rinter)[0] <= F32_TOL
+    assert _err(_np(lse), rlse)[0] <= F32_TOL
+    ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
+    for name, a, b in zip(("dQ", "dK", "dV"), grads, ref):
+        assert _err(_np(a), b)[0] <= F32_TOL, name
+
+
+@pytest.mark.parametrize("grid,tiles,d", [
+    ((4, 22, 40), [(1, 1, 20), (1, 11, 20)], 128),     # 20 | 11 | 16 tokens per group
+    ((2, 44, 40), [(1, 2, 20), (1, 22, 20)], 128),     # 40-token, 11-token, 8-token groups
+    ((80, 8, 8), [(1, 2, 2), (2, 4, 4)], 128),         # last pass: 160-token groups in two boxes
+    ((4, 16, 16), [(1, 4, 4), (2, 8, 8)], 64),         # d = 64
+    ((2, 8, 16), [(1, 1, 2), (1, 2, 4), (2, 4, 8)], 128),  # four passes
+])
+def test_bf16_passes_forward_and_backward(cuda_ok, grid, tiles, d):
+    inp = random_problem(53, 1, 2, d, grid, (1, 1, 1), dtype=torch.bfloat16, k_bias_std=1.0, with_do=True)
+    o, inter, lse, grads = _gpu_fwd_bwd(inp, grid, tiles)
+    ro, rinter, rlse, _ = oracle.squad_fwd_multi(inp.q, inp.k, inp.v, grid, tiles)
+    mx, mean = _err(_np(o), ro)
+    assert mx <= BF16_MAX and mean <= BF16_MEAN, (mx, mean)
+    for j in range(len(tiles)):
+        mx, mean = _err(_np(inter[j]), rinter[j])
+        assert mx <= BF16_MAX and mean <= BF16_MEAN, (j, mx, mean)
+    ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
+    for name, a, b in zip(("dQ", "dK", "dV"), grads, ref):
+        assert np.isfinite(_np(a)).all(), name
+        assert _err(_np(a), b)[0] <= GRAD_MAX, name
+
+
+def test_one_tile_matches_the_two_pass_operator(cuda_ok):
+    grid, tile = (4, 22, 40), (1, 11, 20)
+    inp = random_problem(55, 1, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
+    o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, grid, [tile])
+    o2, o1, l1, l2 = sq.squad_attn_fwd(q, k, v, grid, tile)
+    sq.poll_device_error()
+    assert torch.equal(o, o2) and torch.equal(inter[0], o1)
+    assert torch.equal(lse[0], l1) and torch.equal(lse[1], l2)
+
+
+def test_autograd_through_three_passes(cuda_ok):
+    grid, tiles = (2, 8, 8), [(1, 2, 2), (2, 4, 4)]
+    inp = random_problem(57, 1, 2, 128, grid, (1, 1, 1), dtype=torch.bfloat16, with_do=True)
+    q, k, v = (t.cuda().requires_grad_(True) for t in (inp.q, inp.k, inp.v))
+    o = sq.attention_multi(q, k, v, grid, tiles)
+    o.backward(inp.do.cuda())
+    ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
+    for name, t, r in zip(("dQ", "dK", "dV"), (q, k, v), ref):
+        assert _err(_np(t.grad), r)[0] <= GRAD_MAX, name
+
+
+def test_three_passes_on_the_video_shape(cuda_ok):
+    # the 27,280-token shape with windows of 220 = 20 x 11: groups of 20, 11 and 124 tokens
+    wl = WORKLOADS["wan5b_fwd"]
+    inp = make_inputs(wl)
+    tiles = [(1, 1, 20), (1, 11, 20)]
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    o, _, _ = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles)
+    sq.poll_device_error()
+    for h in (0, 17):
+        sel = (slice(0, 1), slice(h, h + 1))
+        ro, _, _, _ = oracle.squad_fwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, tiles)
+        mx, mean = _err(_np(o[sel]), ro)
+        assert mx <= BF16_MAX and mean <= BF16_MEAN, (h, mx, mean)

@@ -161,12 +161,19 @@ def whole_job_throughput(world: int, flops_per_rank_step: float, ms_per_step: fl
     return world * flops_per_rank_step / (ms_per_step / 1e3) / 1e12
 
 
-def source_sha(path: str) -> str:
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+FWD_KERNEL_SOURCES = ("squad_fwd_tc.cuh", "sm100.cuh", "geometry.h")
 
 
-def read_traffic(kernel_key: str, src_path: str, units_scale: float = 1.0):
+def source_sha(paths) -> str:
+    """First 16 hex digits of the SHA-256 of the concatenated kernel sources."""
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel_key: str, src_paths, units_scale: float = 1.0):
     """DRAM bytes per launch of a kernel from the committed ncu summary, or None when the
     summary is missing or was taken on a different version of the kernel source."""
     prof = os.path.join(ROOT, "profiles", "ncu_fwd_tc_wan5b.md")
@@ -175,7 +182,7 @@ def read_traffic(kernel_key: str, src_path: str, units_scale: float = 1.0):
     text = open(prof).read()
     m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
     m_val = re.search(rf"{kernel_key}_dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_sha or not m_val or m_sha.group(1) != source_sha(src_path):
+    if not m_sha or not m_val or m_sha.group(1) != source_sha(src_paths):
         return None
     return int(m_val.group(1)) * units_scale
 
@@ -361,7 +368,7 @@ def main():
     # on its own reads three [rows, d] tensors and writes one, the same byte count.
     alg_bytes = 4 * rows * wl.d * 2
     pass_flops = {1: 4.0 * rows * wl.d * wl.w, 2: 4.0 * rows * wl.d * wl.m}
-    src = os.path.join(ROOT, "sub_quadratic_two_b200", "csrc", "squad_fwd_tc.cuh")
+    src = [os.path.join(ROOT, "sub_quadratic_two_b200", "csrc", f) for f in FWD_KERNEL_SOURCES]
     achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
     roofline = {
         "bound": "hbm", "kernel": "squad_fwd_tc_kernel (one fused launch per step: local then global pass)",
@@ -478,6 +485,19 @@ def main():
                                           "speedup_of_squad": dms / oms}
             configs[name] = entry
             del oq, okk, ov, oo, ows
+
+        # three passes over nested tiles on the headline inputs: 1x1x20 | 1x11x20 | grid,
+        # groups of 20, 11 and 124 tokens (one launch per pass)
+        tiles3 = [(1, 1, 20), (1, 11, 20)]
+        mms = time_flushed(lambda: sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3), 20)
+        sq.poll_device_error()
+        ratios = [20, 11, wl.n // 220]
+        mflops = 4.0 * wl.B * wl.heads * wl.n * wl.d * sum(ratios)
+        configs["wan5b_fwd_3pass"] = {
+            "ms": mms, "TFLOP/s": mflops / mms / 1e9, "useful_flops": mflops, "tiles": [list(t) for t in tiles3],
+            "group_sizes": ratios, "GB/s_per_pass_floor": 3 * alg_bytes / (mms / 1e3) / 1e9,
+            "timing": "median of 20 calls, L2 flushed before each",
+            "note": "three launches; each pass reads Q, K and its values and writes its output (3 x 670 MB algorithmic)"}
 
     # ---------------- CPU baseline: the oracle on host cores, rank 0 at N=1 only
     cpu = None

@@ -50,13 +50,28 @@ struct Geom {
 };
 
 // Global token index (b,h offset included) of row 0 of problem `prob`.
+// A group of three digits whose extents are all 1 is skipped (the two SQuad passes use
+// one group each), which keeps the divisions off the kernels' scheduling path.
 SQ_HD int problem_base(const Geom& g, int prob) {
   const int bh = prob / g.probs, idx = prob - bh * g.probs;
   const int q0 = g.p0 * g.p1 * g.p2;  // problems per outer window
-  const int in = idx % q0, out = idx / q0;
-  const int i0 = in % g.p0, i1 = (in / g.p0) % g.p1, i2 = in / (g.p0 * g.p1);
-  const int i3 = out % g.p3, i4 = (out / g.p3) % g.p4, i5 = out / (g.p3 * g.p4);
-  return bh * g.n + i0 * g.o0 + i1 * g.o1 + i2 * g.o2 + i3 * g.o3 + i4 * g.o4 + i5 * g.o5;
+  int in = idx, out = 0;
+  if (q0 != g.probs) {
+    out = idx / q0;
+    in = idx - out * q0;
+  }
+  int base = bh * g.n;
+  if (q0 > 1) {
+    const int t = in / g.p0, i0 = in - t * g.p0;
+    const int i2 = t / g.p1, i1 = t - i2 * g.p1;
+    base += i0 * g.o0 + i1 * g.o1 + i2 * g.o2;
+  }
+  if (out > 0) {
+    const int t = out / g.p3, i3 = out - t * g.p3;
+    const int i5 = t / g.p4, i4 = t - i5 * g.p4;
+    base += i3 * g.o3 + i4 * g.o4 + i5 * g.o5;
+  }
+  return base;
 }
 
 // Token offset of row i (0 <= i < L) of a problem, rows ordered (c, b, a).

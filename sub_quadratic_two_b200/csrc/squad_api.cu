@@ -24,8 +24,8 @@ using sq::Geom;
 
 constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr int kMaxDevices = 64;
-constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
-constexpr int kFusedLag = 2;  // see decode_item  // 2 s per wait: far above any legitimate wait
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
+constexpr int kFusedLag = 2;  // heads between a local pass and its global pass (see decode_item)
 
 thread_local int t_last_cuda = 0;
 

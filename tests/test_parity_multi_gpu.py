@@ -1,7 +1,12 @@
 """GPU parity of the k-pass entry points (passes over nested tiles) against the oracle.
 
-Same tolerances as the two-pass operator: fp32 max |err| <= 1e-5; bf16 forward
-max <= 1.5e-2 and mean <= 2e-3; bf16 gradients max <= 3e-2. Reading of the
+fp32: max |err| <= 1e-5, as for the two-pass operator. bf16: the two-pass
+tolerances (forward max 1.5e-2, mean 2e-3; gradients max 3e-2) budget two
+passes, each of which rounds its probabilities to bf16 before the P.V product and
+stores its output in bf16; a pass passes the error of its values on through a
+convex combination, so the errors of k passes add. The bf16 bounds here are
+therefore the two-pass ones times k / 2 (three passes: max 2.25e-2, mean 3e-3;
+gradients 4.5e-2). Reading of the
 pages' outlook on composing more than two passes ("SQuad: Sub-Quadratic
 Attention Distillation for Efficient Video Generation", gist.science technical
 summary, Significance and Claims): nested tiles, pass j attends within a
@@ -18,7 +23,13 @@ from workloads import WORKLOADS, make_inputs, random_problem
 pytestmark = pytest.mark.gpu
 
 F32_TOL = 1e-5
-BF16_MAX, BF16_MEAN, GRAD_MAX = 1.5e-2, 2e-3, 3e-2
+BF16_MAX, BF16_MEAN, GRAD_MAX = 1.5e-2, 2e-3, 3e-2   # two passes
+
+
+def _bf16_tol(npasses):
+    """(forward max, forward mean, gradient max) for npasses bf16 passes."""
+    f = npasses / 2.0
+    return BF16_MAX * f, BF16_MEAN * f, GRAD_MAX * f
 
 
 def _np(t):
@@ -66,15 +77,18 @@ def test_bf16_passes_forward_and_backward(cuda_ok, grid, tiles, d):
     inp = random_problem(53, 1, 2, d, grid, (1, 1, 1), dtype=torch.bfloat16, k_bias_std=1.0, with_do=True)
     o, inter, lse, grads = _gpu_fwd_bwd(inp, grid, tiles)
     ro, rinter, rlse, _ = oracle.squad_fwd_multi(inp.q, inp.k, inp.v, grid, tiles)
+    fmax, fmean, gmax = _bf16_tol(len(tiles) + 1)
     mx, mean = _err(_np(o), ro)
-    assert mx <= BF16_MAX and mean <= BF16_MEAN, (mx, mean)
+    assert mx <= fmax and mean <= fmean, (mx, mean)
     for j in range(len(tiles)):
+        # the output of pass j + 1 carries the rounding of j + 1 passes
+        jmax, jmean, _ = _bf16_tol(max(2, j + 1))
         mx, mean = _err(_np(inter[j]), rinter[j])
-        assert mx <= BF16_MAX and mean <= BF16_MEAN, (j, mx, mean)
+        assert mx <= jmax and mean <= jmean, (j, mx, mean)
     ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
     for name, a, b in zip(("dQ", "dK", "dV"), grads, ref):
         assert np.isfinite(_np(a)).all(), name
-        assert _err(_np(a), b)[0] <= GRAD_MAX, name
+        assert _err(_np(a), b)[0] <= gmax, name
 
 
 def test_one_tile_matches_the_two_pass_operator(cuda_ok):
@@ -95,8 +109,9 @@ def test_autograd_through_three_passes(cuda_ok):
     o = sq.attention_multi(q, k, v, grid, tiles)
     o.backward(inp.do.cuda())
     ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
+    gmax = _bf16_tol(len(tiles) + 1)[2]
     for name, t, r in zip(("dQ", "dK", "dV"), (q, k, v), ref):
-        assert _err(_np(t.grad), r)[0] <= GRAD_MAX, name
+        assert _err(_np(t.grad), r)[0] <= gmax, name
 
 
 def test_three_passes_on_the_video_shape(cuda_ok):
@@ -107,8 +122,9 @@ def test_three_passes_on_the_video_shape(cuda_ok):
     q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
     o, _, _ = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles)
     sq.poll_device_error()
+    fmax, fmean, _ = _bf16_tol(3)
     for h in (0, 17):
         sel = (slice(0, 1), slice(h, h + 1))
         ro, _, _, _ = oracle.squad_fwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, tiles)
         mx, mean = _err(_np(o[sel]), ro)
-        assert mx <= BF16_MAX and mean <= BF16_MEAN, (h, mx, mean)
+        assert mx <= fmax and mean <= fmean, (h, mx, mean)

@@ -23,6 +23,8 @@
 // 128 rows; a tile is a sub-box that is cut along b or along c.
 #pragma once
 
+#include <cstdint>
+
 #ifdef __CUDACC__
 #define SQ_HD __host__ __device__ __forceinline__
 #else
@@ -30,6 +32,37 @@
 #endif
 
 namespace sq {
+
+// Division by a divisor that is fixed for a launch, as a multiply-high, an add and a
+// shift, after the unsigned method of Granlund and Montgomery ("Division by Invariant
+// Integers using Multiplication", PLDI 1994): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, the 33-bit multiplier 2^32 + m gives
+// floor(x / d) = floor((x (2^32 + m)) / 2^(32 + l)) = (umulhi(x, m) + x) >> l for every
+// 0 <= x < 2^32; for x < 2^31 the sum fits in 32 bits. The kernels' scheduling threads
+// decode work indices with it, since a hardware-less integer division is a long
+// dependent chain on their critical path.
+struct FastDiv {
+  uint32_t d;  // divisor, 1 <= d < 2^31
+  uint32_t m;  // multiplier (low 32 bits of 2^32 + m)
+  uint32_t l;  // shift, ceil(log2 d)
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  while ((uint64_t(1) << f.l) < d) ++f.l;
+  f.m = uint32_t(((uint64_t(1) << 32) * ((uint64_t(1) << f.l) - d)) / d + 1);
+  return f;
+}
+
+// floor(x / f.d) for 0 <= x < 2^31.
+SQ_HD int fdiv(int x, const FastDiv& f) {
+#ifdef __CUDA_ARCH__
+  const uint32_t hi = __umulhi(uint32_t(x), f.m);
+#else
+  const uint32_t hi = uint32_t((uint64_t(uint32_t(x)) * f.m) >> 32);
+#endif
+  return int((hi + uint32_t(x)) >> f.l);
+}
 
 struct Geom {
   int a_n, b_n, c_n;  // problem box extents
@@ -47,28 +80,31 @@ struct Geom {
   int nb;             // tiles along b
   int nt;             // tiles per problem
   int box_rows;       // a_n * b_sub * c_sub
+  // the divisors above as FastDiv (q0 = p0 p1 p2, problems per outer window)
+  FastDiv f_probs, f_q0, f_p0, f_p1, f_p3, f_p4, f_an, f_bn;
+  FastDiv f_bsub, f_nb, f_nt;  // set with the tiling
 };
 
 // Global token index (b,h offset included) of row 0 of problem `prob`.
 // A group of three digits whose extents are all 1 is skipped (the two SQuad passes use
 // one group each), which keeps the divisions off the kernels' scheduling path.
 SQ_HD int problem_base(const Geom& g, int prob) {
-  const int bh = prob / g.probs, idx = prob - bh * g.probs;
+  const int bh = fdiv(prob, g.f_probs), idx = prob - bh * g.probs;
   const int q0 = g.p0 * g.p1 * g.p2;  // problems per outer window
   int in = idx, out = 0;
   if (q0 != g.probs) {
-    out = idx / q0;
+    out = fdiv(idx, g.f_q0);
     in = idx - out * q0;
   }
   int base = bh * g.n;
   if (q0 > 1) {
-    const int t = in / g.p0, i0 = in - t * g.p0;
-    const int i2 = t / g.p1, i1 = t - i2 * g.p1;
+    const int t = fdiv(in, g.f_p0), i0 = in - t * g.p0;
+    const int i2 = fdiv(t, g.f_p1), i1 = t - i2 * g.p1;
     base += i0 * g.o0 + i1 * g.o1 + i2 * g.o2;
   }
   if (out > 0) {
-    const int t = out / g.p3, i3 = out - t * g.p3;
-    const int i5 = t / g.p4, i4 = t - i5 * g.p4;
+    const int t = fdiv(out, g.f_p3), i3 = out - t * g.p3;
+    const int i5 = fdiv(t, g.f_p4), i4 = t - i5 * g.p4;
     base += i3 * g.o3 + i4 * g.o4 + i5 * g.o5;
   }
   return base;
@@ -76,14 +112,16 @@ SQ_HD int problem_base(const Geom& g, int prob) {
 
 // Token offset of row i (0 <= i < L) of a problem, rows ordered (c, b, a).
 SQ_HD int row_offset(const Geom& g, int i) {
-  const int a = i % g.a_n, b = (i / g.a_n) % g.b_n, c = i / (g.a_n * g.b_n);
+  const int t = fdiv(i, g.f_an), a = i - t * g.a_n;
+  const int c = fdiv(t, g.f_bn), b = t - c * g.b_n;
   return a * g.sA + b * g.sB + c * g.sC;
 }
 
 // First b and c coordinate of tile t.
 SQ_HD void tile_origin(const Geom& g, int t, int& b0, int& c0) {
-  b0 = (t % g.nb) * g.b_sub;
-  c0 = (t / g.nb) * g.c_sub;
+  const int q = fdiv(t, g.f_nb);
+  b0 = (t - q * g.nb) * g.b_sub;
+  c0 = q * g.c_sub;
 }
 
 // Rows of tile t that lie inside the problem; they are a prefix of the tile.
@@ -99,7 +137,8 @@ SQ_HD int tile_valid_rows(const Geom& g, int t) {
 SQ_HD int tile_row_offset(const Geom& g, int t, int i) {
   int b0, c0;
   tile_origin(g, t, b0, c0);
-  const int a = i % g.a_n, bb = (i / g.a_n) % g.b_sub, cc = i / (g.a_n * g.b_sub);
+  const int r = fdiv(i, g.f_an), a = i - r * g.a_n;
+  const int cc = fdiv(r, g.f_bsub), bb = r - cc * g.b_sub;
   return a * g.sA + (b0 + bb) * g.sB + (c0 + cc) * g.sC;
 }
 
@@ -124,6 +163,9 @@ inline bool plan_tiles(Geom& g, int max_rows = 128) {
     g.nt = g.nb * g.c_n;
   }
   g.box_rows = g.a_n * g.b_sub * g.c_sub;
+  g.f_bsub = make_fastdiv(uint32_t(g.b_sub));
+  g.f_nb = make_fastdiv(uint32_t(g.nb));
+  g.f_nt = make_fastdiv(uint32_t(g.nt));
   return true;
 }
 
@@ -142,6 +184,14 @@ inline Geom make_geom_pass(int B, int heads, int T, int H, int W, int iT, int iH
   g.o3 = cW; g.o4 = cH * W; g.o5 = cT * H * W;
   g.probs = g.p0 * g.p1 * g.p2 * g.p3 * g.p4 * g.p5;
   g.L = g.a_n * g.b_n * g.c_n;
+  g.f_probs = make_fastdiv(uint32_t(g.probs));
+  g.f_q0 = make_fastdiv(uint32_t(g.p0 * g.p1 * g.p2));
+  g.f_p0 = make_fastdiv(uint32_t(g.p0));
+  g.f_p1 = make_fastdiv(uint32_t(g.p1));
+  g.f_p3 = make_fastdiv(uint32_t(g.p3));
+  g.f_p4 = make_fastdiv(uint32_t(g.p4));
+  g.f_an = make_fastdiv(uint32_t(g.a_n));
+  g.f_bn = make_fastdiv(uint32_t(g.b_n));
   return g;
 }
 

@@ -237,6 +237,9 @@ squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, cons
   a.bh = p.g1.bh;
   a.lag = kFusedLag < a.bh ? kFusedLag : a.bh;
   a.total_items = (do1 ? a.bh * a.ps[0].pairs_per_bh : 0) + (do2 ? a.bh * a.ps[1].pairs_per_bh : 0);
+  a.f_n1 = sq::make_fastdiv(uint32_t(a.ps[0].pairs_per_bh));
+  a.f_n2 = sq::make_fastdiv(uint32_t(a.ps[1].pairs_per_bh));
+  a.f_n12 = sq::make_fastdiv(uint32_t(a.ps[0].pairs_per_bh + a.ps[1].pairs_per_bh));
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.counters = counters;
   a.discard_base = static_cast<const uint8_t*>(discard);

@@ -380,7 +380,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
       };
       bool ok = true;
       for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
-        const int prob = item / nt, kb = item - prob * nt;
+        const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
         const int base = problem_base(g, prob);
         for (int qb = 0; qb < nt; ++qb) {
           const SlotPlan::Rec r = plan.next(qb == 0, qb == nt - 1);
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
-      const int prob = item / nt, kb = item - prob * nt;
+      const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
       const int base = problem_base(g, prob);
       const bool rlive = row < tile_valid_rows(g, kb);
       for (int qb = 0; qb < nt; ++qb, ++t) {
@@ -587,7 +587,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     uint32_t i = 0, t = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x, ++i) {
-      const int prob = item / nt, kb = item - prob * nt;
+      const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
       const int base = problem_base(g, prob);
       for (int qb = 0; qb < nt; ++qb, ++t) {
         const bool liveq = row < tile_valid_rows(g, qb);

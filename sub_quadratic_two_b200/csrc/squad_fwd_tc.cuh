@@ -57,6 +57,7 @@ struct FwdArgs {
   int bh;                        // batch * heads
   int lag;                       // FWD_FUSED: heads between a head's local pass and its global pass
   int total_items;               // pairs over all (batch, head) and passes run
+  FastDiv f_n1, f_n2, f_n12;     // ps[0].pairs_per_bh, ps[1].pairs_per_bh and their sum
   float scale_log2;              // softmax scale * log2(e)
   uint32_t* counters;            // FWD_FUSED: finished local-pass jobs per (batch, head)
   const uint8_t* discard_base;   // FWD_FUSED inference: local-pass output to drop from L2, or nullptr
@@ -98,14 +99,23 @@ struct Item {
 // still in L2.
 __device__ __forceinline__ Item decode_item(const FwdArgs& a, int i) {
   const int n1 = a.ps[0].pairs_per_bh, n2 = a.ps[1].pairs_per_bh;
-  if (a.mode == FWD_LOCAL) return {0, i / n1, i % n1};
-  if (a.mode == FWD_GLOBAL) return {1, i / n2, i % n2};
+  if (a.mode == FWD_LOCAL) {
+    const int q = fdiv(i, a.f_n1);
+    return {0, q, i - q * n1};
+  }
+  if (a.mode == FWD_GLOBAL) {
+    const int q = fdiv(i, a.f_n2);
+    return {1, q, i - q * n2};
+  }
   const int lag = a.lag;
-  if (i < lag * n1) return {0, i / n1, i % n1};
-  const int j = i - lag * n1, blk = j / (n1 + n2), r = j - blk * (n1 + n2);
+  if (i < lag * n1) {
+    const int q = fdiv(i, a.f_n1);
+    return {0, q, i - q * n1};
+  }
+  const int j = i - lag * n1, blk = fdiv(j, a.f_n12), r = j - blk * (n1 + n2);
   if (blk < a.bh - lag) return r < n1 ? Item{0, blk + lag, r} : Item{1, blk, r - n1};
-  const int t = j - (a.bh - lag) * (n1 + n2);
-  return {1, a.bh - lag + t / n2, t % n2};
+  const int t = j - (a.bh - lag) * (n1 + n2), q = fdiv(t, a.f_n2);
+  return {1, a.bh - lag + q, t - q * n2};
 }
 
 struct Job {
@@ -120,7 +130,7 @@ __device__ __forceinline__ Job job_of(const FwdArgs& a, const Item& it, int whic
   const int j = 2 * it.pair + which;
   Job jb;
   jb.valid = j < p.jobs_per_bh;
-  const int pl = j / p.g.nt;
+  const int pl = fdiv(j, p.g.f_nt);
   jb.qt = j - pl * p.g.nt;
   jb.prob = it.bh * p.g.probs + pl;
   jb.base = jb.valid ? problem_base(p.g, jb.prob) : 0;

@@ -152,11 +152,15 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
  * the position inside their t_{j-1}-window (t_0 = one token, t_k = the grid);
  * its values are the output of pass j-1 (v for j = 1); q, k and the scale are
  * those of every pass; the result is the output of pass k. ntiles = 1 is
- * squad_attn_fwd with tile t_1. Cost: 4 n d (|t_1| + |t_2|/|t_1| + ... +
- * n/|t_{k-1}|) FLOPs per (batch, head). Each pass is one launch of the
- * kernels above (no fused hand-off between passes). On bf16 every pass's box
- * row (t_j / t_{j-1} along W) must be at most 128 tokens (else
- * SQUAD_ERR_UNSUPPORTED); tiles that do not nest give SQUAD_ERR_SHAPE. */
+ * the operator of squad_attn_fwd with tile t_1. Cost: 4 n d (|t_1| +
+ * |t_2|/|t_1| + ... + n/|t_{k-1}|) FLOPs per (batch, head). Each pass is one
+ * launch of the kernels above (no fused hand-off between passes). On bf16 the
+ * forward packs the problems of a pass several to a tensor-core box when they
+ * have at most 64 tokens and the problem box has an extent-1 dimension (a
+ * per-row key mask keeps them apart); the results then equal the unpacked
+ * ones up to fp32 summation order. On bf16 every pass's box row (t_j / t_{j-1}
+ * along W) must be at most 128 tokens (else SQUAD_ERR_UNSUPPORTED); tiles
+ * that do not nest give SQUAD_ERR_SHAPE. */
 
 /* Forward. inter: ntiles consecutive [B, heads, n, d] tensors of the input
  * dtype receiving the outputs of passes 1..k-1 (required: each is the next

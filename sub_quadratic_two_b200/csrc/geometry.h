@@ -21,6 +21,12 @@
 // six digits. The two passes above are j = 1 and j = 2 of k = 2.
 // The tensor-core kernels move a problem through TMA boxes ("tiles") of at most
 // 128 rows; a tile is a sub-box that is cut along b or along c.
+// Packing (forward only): problems of at most 64 rows leave most of a 128-row
+// tensor-core tile empty. When one box dimension has extent 1, P problems that are
+// consecutive along one problem digit share a box instead: that box dimension runs
+// along the digit (stride and tensor-map extent of the digit), the digit's extent
+// shrinks to the number of groups, and a key column belongs to the same problem as
+// a query row when the two sit at the same position along that dimension.
 #pragma once
 
 #include <cstdint>
@@ -83,12 +89,19 @@ struct Geom {
   // the divisors above as FastDiv (q0 = p0 p1 p2, problems per outer window)
   FastDiv f_probs, f_q0, f_p0, f_p1, f_p3, f_p4, f_an, f_bn;
   FastDiv f_bsub, f_nb, f_nt;  // set with the tiling
+  // packing (plan_pack): pk problems per box along box dimension pk_dim (0 a, 1 b, 2 c;
+  // -1: none) and problem digit pk_digit (0..5), whose extent was pk_ext and token
+  // offset pk_stride; pk_rowdiv rows separate neighbouring packed problems in a box
+  int pk, pk_dim, pk_digit, pk_ext, pk_stride, pk_rowdiv;
+  FastDiv f_pk, f_pkrow;
 };
 
-// Global token index (b,h offset included) of row 0 of problem `prob`.
-// A group of three digits whose extents are all 1 is skipped (the two SQuad passes use
-// one group each), which keeps the divisions off the kernels' scheduling path.
-SQ_HD int problem_base(const Geom& g, int prob) {
+// Global token index (b,h offset included) of row 0 of problem `prob`; for a packed
+// geometry also the position j0 of its first problem along the packed digit (the
+// returned base includes j0 * pk_stride). A group of three digits whose extents are
+// all 1 is skipped (the two SQuad passes use one group each), which keeps the
+// divisions off the kernels' scheduling path.
+SQ_HD int problem_base(const Geom& g, int prob, int* j0 = nullptr) {
   const int bh = fdiv(prob, g.f_probs), idx = prob - bh * g.probs;
   const int q0 = g.p0 * g.p1 * g.p2;  // problems per outer window
   int in = idx, out = 0;
@@ -97,17 +110,34 @@ SQ_HD int problem_base(const Geom& g, int prob) {
     in = idx - out * q0;
   }
   int base = bh * g.n;
+  int dig[6] = {0, 0, 0, 0, 0, 0};
   if (q0 > 1) {
-    const int t = fdiv(in, g.f_p0), i0 = in - t * g.p0;
-    const int i2 = fdiv(t, g.f_p1), i1 = t - i2 * g.p1;
-    base += i0 * g.o0 + i1 * g.o1 + i2 * g.o2;
+    const int t = fdiv(in, g.f_p0);
+    dig[0] = in - t * g.p0;
+    dig[2] = fdiv(t, g.f_p1);
+    dig[1] = t - dig[2] * g.p1;
+    base += dig[0] * g.o0 + dig[1] * g.o1 + dig[2] * g.o2;
   }
   if (out > 0) {
-    const int t = fdiv(out, g.f_p3), i3 = out - t * g.p3;
-    const int i5 = fdiv(t, g.f_p4), i4 = t - i5 * g.p4;
-    base += i3 * g.o3 + i4 * g.o4 + i5 * g.o5;
+    const int t = fdiv(out, g.f_p3);
+    dig[3] = out - t * g.p3;
+    dig[5] = fdiv(t, g.f_p4);
+    dig[4] = t - dig[5] * g.p4;
+    base += dig[3] * g.o3 + dig[4] * g.o4 + dig[5] * g.o5;
+  }
+  if (j0 != nullptr) {
+    const int q = g.pk_digit;
+    *j0 = g.pk_dim < 0 ? 0
+                       : (q == 0 ? dig[0] : q == 1 ? dig[1] : q == 2 ? dig[2] : q == 3 ? dig[3] : q == 4 ? dig[4] : dig[5]) *
+                             g.pk;
   }
   return base;
+}
+
+// Packed geometry: the position (0 <= id < pk) of box row i along the packed dimension.
+SQ_HD int pack_id(const Geom& g, int i) {
+  const int t = fdiv(i, g.f_pkrow);
+  return t - fdiv(t, g.f_pk) * g.pk;
 }
 
 // Token offset of row i (0 <= i < L) of a problem, rows ordered (c, b, a).
@@ -192,7 +222,70 @@ inline Geom make_geom_pass(int B, int heads, int T, int H, int W, int iT, int iH
   g.f_p4 = make_fastdiv(uint32_t(g.p4));
   g.f_an = make_fastdiv(uint32_t(g.a_n));
   g.f_bn = make_fastdiv(uint32_t(g.b_n));
+  g.pk = 1;
+  g.pk_dim = -1;
+  g.pk_digit = 0;
+  g.pk_ext = 1;
+  g.pk_stride = 0;
+  g.pk_rowdiv = 1;
+  g.f_pk = make_fastdiv(1u);
+  g.f_pkrow = make_fastdiv(1u);
   return g;
+}
+
+// Pack several problems into one box when a problem has at most max_rows / 2 rows and
+// a box dimension has extent 1 (see the packing note at the top). The slowest such
+// dimension is used (c, then b, then a), along the problem digit that fills the box
+// best; groups are balanced (the digit's extent p is cut into ceil(p / P) groups of at
+// most P problems). Call before plan_tiles. Returns whether the geometry was packed.
+inline bool plan_pack(Geom& g, int max_rows = 128) {
+  if (2 * g.L > max_rows) return false;
+  const int dim = g.c_n == 1 ? 2 : g.b_n == 1 ? 1 : g.a_n == 1 ? 0 : -1;
+  if (dim < 0) return false;
+  int* ext[6] = {&g.p0, &g.p1, &g.p2, &g.p3, &g.p4, &g.p5};
+  int* off[6] = {&g.o0, &g.o1, &g.o2, &g.o3, &g.o4, &g.o5};
+  const int cap = max_rows / g.L;
+  int q = -1, best = 1;
+  for (int i = 0; i < 6; ++i) {
+    const int fill = *ext[i] < cap ? *ext[i] : cap;
+    if (fill > best) {
+      best = fill;
+      q = i;
+    }
+  }
+  if (q < 0) return false;
+  const int p = *ext[q], groups = ceil_div(p, best), P = ceil_div(p, groups);
+  g.pk = P;
+  g.pk_dim = dim;
+  g.pk_digit = q;
+  g.pk_ext = p;
+  g.pk_stride = *off[q];
+  if (dim == 0) {
+    g.a_n = P;
+    g.sA = g.pk_stride;
+  } else if (dim == 1) {
+    g.b_n = P;
+    g.sB = g.pk_stride;
+  } else {
+    g.c_n = P;
+    g.sC = g.pk_stride;
+  }
+  g.pk_rowdiv = dim == 0 ? 1 : dim == 1 ? g.a_n : g.a_n * g.b_n;
+  g.probs = g.probs / p * groups;
+  *ext[q] = groups;
+  *off[q] = g.pk_stride * P;
+  g.L = g.a_n * g.b_n * g.c_n;
+  g.f_probs = make_fastdiv(uint32_t(g.probs));
+  g.f_q0 = make_fastdiv(uint32_t(g.p0 * g.p1 * g.p2));
+  g.f_p0 = make_fastdiv(uint32_t(g.p0));
+  g.f_p1 = make_fastdiv(uint32_t(g.p1));
+  g.f_p3 = make_fastdiv(uint32_t(g.p3));
+  g.f_p4 = make_fastdiv(uint32_t(g.p4));
+  g.f_an = make_fastdiv(uint32_t(g.a_n));
+  g.f_bn = make_fastdiv(uint32_t(g.b_n));
+  g.f_pk = make_fastdiv(uint32_t(P));
+  g.f_pkrow = make_fastdiv(uint32_t(g.pk_rowdiv));
+  return true;
 }
 
 // stage 1 = local (window) pass, stage 2 = global (cross-window) pass.

@@ -157,7 +157,10 @@ BwdWs bwd_workspace(const Plan& p, const squad_desc* d) {
 // token strides; boxes of (64, a_n, b_sub, c_sub, 1), 128-byte swizzle.
 squad_status encode_map(CUtensorMap* m, const void* base, const Geom& g, int d, long long rows) {
   const cuuint64_t esz = 2;
-  cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(g.a_n), cuuint64_t(g.b_n), cuuint64_t(g.c_n), cuuint64_t(rows)};
+  // a packed dimension spans the packed digit's full extent (its rows past that extent read as zeros)
+  cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(g.pk_dim == 0 ? g.pk_ext : g.a_n),
+                        cuuint64_t(g.pk_dim == 1 ? g.pk_ext : g.b_n), cuuint64_t(g.pk_dim == 2 ? g.pk_ext : g.c_n),
+                        cuuint64_t(rows)};
   cuuint64_t strides[4] = {cuuint64_t(g.sA) * d * esz, cuuint64_t(g.sB) * d * esz, cuuint64_t(g.sC) * d * esz,
                            cuuint64_t(d) * esz};
   cuuint32_t box[5] = {64u, cuuint32_t(g.a_n), cuuint32_t(g.b_sub), cuuint32_t(g.c_sub), 1u};
@@ -693,6 +696,7 @@ struct MultiPlan {
   Plan base;                 // scale, rows, element size (its g1/g2 are unused)
   int k;                     // passes
   Geom g[kMaxTiles + 1];     // pass j at g[j - 1]
+  Geom gf[kMaxTiles + 1];    // the same for the bf16 forward, small problems packed several to a box
 };
 
 squad_status make_multi_plan(const squad_desc* d, int ntiles, const int* tiles, MultiPlan* mp) {
@@ -713,8 +717,14 @@ squad_status make_multi_plan(const squad_desc* d, int ntiles, const int* tiles, 
       if (in[a] <= 0 || out[a] <= 0 || out[a] % in[a] != 0 || grid[a] % out[a] != 0) return SQUAD_ERR_SHAPE;
     }
     Geom g = sq::make_geom_pass(d->B, d->heads, d->T, d->H, d->W, in[0], in[1], in[2], out[0], out[1], out[2]);
-    if (d->dtype == SQUAD_BF16 && !sq::plan_tiles(g)) return SQUAD_ERR_UNSUPPORTED;
+    Geom gf = g;
+    if (d->dtype == SQUAD_BF16) {
+      if (!sq::plan_tiles(g)) return SQUAD_ERR_UNSUPPORTED;
+      sq::plan_pack(gf);
+      if (!sq::plan_tiles(gf)) return SQUAD_ERR_UNSUPPORTED;
+    }
     mp->g[j - 1] = g;
+    mp->gf[j - 1] = gf;
   }
   return SQUAD_OK;
 }
@@ -795,7 +805,7 @@ squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int*
     float* l = lse == nullptr ? nullptr : lse + size_t(mp.base.rows) * (j - 1);
     if (desc->dtype == SQUAD_BF16) {
       Plan p = mp.base;
-      p.g1 = p.g2 = mp.g[j - 1];
+      p.g1 = p.g2 = mp.gf[j - 1];
       s = launch_fwd_tc(ds, desc->d, sq::FWD_LOCAL, p, q, k, val, out, l, val, out, l, nullptr, nullptr, st);
     } else {
       s = simt_fwd<float>(mp.g[j - 1], q, k, val, out, l, desc->d, mp.base.scale, st);

@@ -123,7 +123,19 @@ struct Job {
   int qt;    // query box within the problem
   int prob;  // problem index over all (batch, head)
   int base;  // first token of the problem
+  int j0;    // packed geometry: position of its first problem along the packed digit
 };
+
+// TMA coordinates (a, b, c, token) of the box of job J whose tile origin is (b0, c0). For
+// a packed geometry the packed dimension starts at j0, so that the tensor map's bound on
+// that dimension (the digit's extent) zero-fills the rows of a short last group.
+__device__ __forceinline__ void box_coords(const Geom& g, const Job& J, int b0, int c0, int& ca, int& cb, int& cc,
+                                           int& ct) {
+  ca = g.pk_dim == 0 ? J.j0 : 0;
+  cb = b0 + (g.pk_dim == 1 ? J.j0 : 0);
+  cc = c0 + (g.pk_dim == 2 ? J.j0 : 0);
+  ct = J.base - J.j0 * g.pk_stride;
+}
 
 __device__ __forceinline__ Job job_of(const FwdArgs& a, const Item& it, int which) {
   const PassArgs& p = a.ps[it.pass];
@@ -133,7 +145,8 @@ __device__ __forceinline__ Job job_of(const FwdArgs& a, const Item& it, int whic
   const int pl = fdiv(j, p.g.f_nt);
   jb.qt = j - pl * p.g.nt;
   jb.prob = it.bh * p.g.probs + pl;
-  jb.base = jb.valid ? problem_base(p.g, jb.prob) : 0;
+  jb.j0 = 0;
+  jb.base = jb.valid ? problem_base(p.g, jb.prob, &jb.j0) : 0;
   return jb;
 }
 
@@ -265,21 +278,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               const uint32_t s = qc % 2;
               if (!(ok = mbar_wait(&bars[F_QE + s], ((qc / 2) & 1) ^ 1, abort_flag, to))) break;
               tile_origin(g, J[x].qt, b0, c0);
+              int ca, cb, cc, ct;
+              box_coords(g, J[x], b0, c0, ca, cb, cc, ct);
               mbar_arrive_expect_tx(&bars[F_QF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d_hint(smem + Lay::Q_OFF + s * Lay::TILE + dh * kBlk, mq, &bars[F_QF + s], dh * 64, 0, b0,
-                                 c0, J[x].base, pol_qk);
+                tma_load_5d_hint(smem + Lay::Q_OFF + s * Lay::TILE + dh * kBlk, mq, &bars[F_QF + s], dh * 64, ca, cb,
+                                 cc, ct, pol_qk);
               ++qc;
             }
             if (x == 1 && shared) continue;
             tile_origin(g, k, b0, c0);
+            int ca, cb, cc, ct;
+            box_coords(g, J[x], b0, c0, ca, cb, cc, ct);
             {
               const uint32_t s = uc % Lay::NKV;
               if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
               mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KVF + s], dh * 64, 0, b0,
-                                 c0, J[x].base, pol_qk);
+                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mk, &bars[F_KVF + s], dh * 64, ca, cb,
+                                 cc, ct, pol_qk);
               ++uc;
             }
             if (!dep_done) {
@@ -294,8 +311,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!(ok = mbar_wait(&bars[F_KVE + s], ((uc / Lay::NKV) & 1) ^ 1, abort_flag, to))) break;
               mbar_arrive_expect_tx(&bars[F_KVF + s], tx);
               for (int dh = 0; dh < DH; ++dh)
-                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_KVF + s], dh * 64, 0, b0,
-                                 c0, J[x].base, pol_v);
+                tma_load_5d_hint(smem + Lay::KV_OFF + s * Lay::TILE + dh * kBlk, mv, &bars[F_KVF + s], dh * 64, ca, cb,
+                                 cc, ct, pol_v);
               ++uc;
             }
           }
@@ -420,6 +437,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int qt;    // query box within the problem
       int base;  // first token of the problem
       int tok;   // this thread's output row, or -1 past the box's valid rows
+      uint64_t mlo, mhi;  // packed geometry: key columns of this row's problem (bits 0-63, 64-127)
     };
     auto find_job = [&](int i) -> SJob {
       for (; i < args.total_items; i += gridDim.x) {
@@ -427,10 +445,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const Job J = job_of(args, it, a);
         if (!J.valid) continue;
         const Geom& g = args.ps[it.pass].g;
-        const int tok = row < tile_valid_rows(g, J.qt) ? J.base + tile_row_offset(g, J.qt, row) : -1;
-        return SJob{i, it.pass, J.qt, J.base, tok};
+        int tok = row < tile_valid_rows(g, J.qt) ? J.base + tile_row_offset(g, J.qt, row) : -1;
+        uint64_t mlo = ~0ull, mhi = ~0ull;
+        if (g.pk > 1) {
+          // the columns at this row's position along the packed dimension: runs of pk_rowdiv
+          // columns, one every pk * pk_rowdiv
+          const int id = pack_id(g, row), R = g.pk_rowdiv;
+          if (J.j0 + id >= g.pk_ext) tok = -1;  // past the digit's extent: zero-filled row
+          mlo = 0ull;
+          mhi = 0ull;
+          for (int s0 = id * R; s0 < 128; s0 += g.pk * R) {
+            const int e = s0 + R < 128 ? s0 + R : 128;
+            if (s0 < 64) {
+              const int e0 = e < 64 ? e : 64;
+              mlo |= (e0 - s0 >= 64 ? ~0ull : ((1ull << (e0 - s0)) - 1ull)) << s0;
+            }
+            if (e > 64) {
+              const int s1 = s0 > 64 ? s0 - 64 : 0, e1 = e - 64;
+              mhi |= (e1 - s1 >= 64 ? ~0ull : ((1ull << (e1 - s1)) - 1ull)) << s1;
+            }
+          }
+        }
+        return SJob{i, it.pass, J.qt, J.base, tok, mlo, mhi};
       }
-      return SJob{args.total_items, 0, 0, 0, -1};
+      return SJob{args.total_items, 0, 0, 0, -1, ~0ull, ~0ull};
     };
     SJob cur = find_job(blockIdx.x);
     while (ok && cur.i < args.total_items) {
@@ -452,6 +490,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 32; ++e)
               if (32 * j + e >= lim) r[32 * j + e] = 0xff800000u;
           }
+        }
+        if (g.pk > 1) {  // packed problems: keys of other problems in the box -> -inf
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (!(((e < 64 ? cur.mlo : cur.mhi) >> (e & 63)) & 1ull)) r[e] = 0xff800000u;
         }
         // row maximum: 8 independent partial maxima of three-input max
         float mp[8];

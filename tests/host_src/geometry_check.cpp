@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <random>
+#include <vector>
 
 using namespace sq;
 
@@ -20,7 +21,7 @@ int main() {
   // FastDiv: every divisor up to 4096 against many numerators, then random large divisors
   for (uint32_t d = 1; d <= 4096; ++d) {
     const FastDiv f = make_fastdiv(d);
-    for (int x = 0; x < 20000; ++x) {
+    for (int x = 0; x < 10000; ++x) {
       if (fdiv(x, f) != int(uint32_t(x) / d)) return fail("fdiv small", x, d, fdiv(x, f));
       ++checked;
     }
@@ -50,7 +51,7 @@ int main() {
       if (n % v == 0) c[k++] = v;
     return c[rng() % k];
   };
-  for (int it = 0; it < 4000; ++it) {
+  for (int it = 0; it < 1500; ++it) {
     const int T = divs[rng() % 9] * divs[rng() % 9], H = divs[rng() % 9] * divs[rng() % 9];
     const int W = divs[rng() % 9] * divs[rng() % 9];
     const int cT = pick(T), cH = pick(H), cW = pick(W);
@@ -82,6 +83,58 @@ int main() {
       }
     }
   }
+  // packing: every packed box row maps, through the tensor map's view, to the token of
+  // exactly one row of one original problem, rows of a problem share their pack_id, and
+  // rows past the packed digit's extent are exactly the out-of-bounds ones
+  int packed_geoms = 0;
+  for (int it = 0; it < 1000; ++it) {
+    const int T = divs[rng() % 9] * divs[rng() % 9], H = divs[rng() % 9] * divs[rng() % 9];
+    const int W = divs[rng() % 9] * divs[rng() % 9];
+    const int cT = pick(T), cH = pick(H), cW = pick(W);
+    const int iT = pick(cT), iH = pick(cH), iW = pick(cW);
+    const Geom u = make_geom_pass(2, 3, T, H, W, iT, iH, iW, cT, cH, cW);
+    Geom g = u;
+    if (!plan_pack(g)) continue;
+    if (!plan_tiles(g)) return fail("plan_tiles after pack", it, g.L, 0);
+    if (g.nt != 1 || g.box_rows != g.L || g.L > 128) return fail("packed tiling", g.nt, g.box_rows, g.L);
+    ++packed_geoms;
+    // owner[token] = (original problem) from the unpacked geometry
+    const int rows = u.bh * u.n;
+    std::vector<int> owner(rows, -1), seen(rows, 0);
+    for (int p = 0; p < u.bh * u.probs; ++p)
+      for (int i = 0; i < u.L; ++i) owner[problem_base(u, p) + row_offset(u, i)] = p;
+    const int mext[3] = {g.pk_dim == 0 ? g.pk_ext : g.a_n, g.pk_dim == 1 ? g.pk_ext : g.b_n,
+                         g.pk_dim == 2 ? g.pk_ext : g.c_n};
+    for (int p = 0; p < g.bh * g.probs; ++p) {
+      int j0 = -1;
+      const int base = problem_base(g, p, &j0);
+      const int tbase = base - j0 * g.pk_stride;
+      if (j0 < 0 || j0 >= g.pk_ext || tbase < 0) return fail("pack origin", p, j0, tbase);
+      const int co[3] = {g.pk_dim == 0 ? j0 : 0, g.pk_dim == 1 ? j0 : 0, g.pk_dim == 2 ? j0 : 0};
+      int id_owner[128];
+      for (int k = 0; k < 128; ++k) id_owner[k] = -1;
+      for (int i = 0; i < g.box_rows; ++i) {
+        const int a = i % g.a_n, b = (i / g.a_n) % g.b_n, c = i / (g.a_n * g.b_n);
+        const bool inb = co[0] + a < mext[0] && co[1] + b < mext[1] && co[2] + c < mext[2];
+        const int id = pack_id(g, i);
+        const int refid = g.pk_dim == 0 ? a : g.pk_dim == 1 ? b : c;
+        if (id != refid) return fail("pack_id", i, id, refid);
+        const bool valid = j0 + id < g.pk_ext;
+        if (valid != inb) return fail("pack validity", p, i, valid);
+        if (!valid) continue;
+        const int tok = base + tile_row_offset(g, 0, i);
+        const int tma = tbase + (co[0] + a) * g.sA + (co[1] + b) * g.sB + (co[2] + c) * g.sC;
+        if (tok != tma || tok < 0 || tok >= rows) return fail("pack token", p, i, tok);
+        if (id_owner[id] < 0) id_owner[id] = owner[tok];
+        if (owner[tok] != id_owner[id]) return fail("pack grouping", p, i, tok);
+        ++seen[tok];
+        ++checked;
+      }
+    }
+    for (int t = 0; t < rows; ++t)
+      if (seen[t] != 1) return fail("pack coverage", it, t, seen[t]);
+  }
+  if (packed_geoms < 50) return fail("too few packed geometries", packed_geoms, 0, 0);
   std::printf("ok %lld\n", checked);
   return 0;
 }

@@ -72,6 +72,9 @@ def test_fp32_passes_forward_and_backward(cuda_ok, grid, tiles, d):
     ((80, 8, 8), [(1, 2, 2), (2, 4, 4)], 128),         # last pass: 160-token groups in two boxes
     ((4, 16, 16), [(1, 4, 4), (2, 8, 8)], 64),         # d = 64
     ((2, 8, 16), [(1, 1, 2), (1, 2, 4), (2, 4, 8)], 128),  # four passes
+    # small problems packed several to a box, along each box dimension, ragged last groups:
+    ((4, 22, 40), [(1, 1, 20), (2, 11, 20)], 128),     # pass 2: 22-token groups packed along a (5 per box)
+    ((4, 22, 40), [(2, 1, 20), (2, 11, 20)], 128),     # pass 1: 40-token windows packed along b (3 per box, 22 = 7 x 3 + 1)
 ])
 def test_bf16_passes_forward_and_backward(cuda_ok, grid, tiles, d):
     inp = random_problem(53, 1, 2, d, grid, (1, 1, 1), dtype=torch.bfloat16, k_bias_std=1.0, with_do=True)
@@ -92,7 +95,9 @@ def test_bf16_passes_forward_and_backward(cuda_ok, grid, tiles, d):
 
 
 def test_one_tile_matches_the_two_pass_operator(cuda_ok):
-    grid, tile = (4, 22, 40), (1, 11, 20)
+    # 220-token windows and 80-token groups: neither pass is packed, so the k-pass
+    # forward runs exactly the two-pass operator's boxes
+    grid, tile = (20, 22, 40), (1, 11, 20)
     inp = random_problem(55, 1, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
     q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.do))
     o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, grid, [tile])
@@ -100,6 +105,24 @@ def test_one_tile_matches_the_two_pass_operator(cuda_ok):
     sq.poll_device_error()
     assert torch.equal(o, o2) and torch.equal(inter[0], o1)
     assert torch.equal(lse[0], l1) and torch.equal(lse[1], l2)
+
+
+def test_one_tile_packed_global_pass(cuda_ok):
+    # 16-token groups: the k-pass forward packs eight of them into a box (the two-pass
+    # operator does not), so both are compared with the oracle
+    grid, tile = (4, 22, 40), (1, 11, 20)
+    inp = random_problem(56, 1, 2, 128, grid, tile, dtype=torch.bfloat16, with_do=True)
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, grid, [tile])
+    o2, o1, l1, l2 = sq.squad_attn_fwd(q, k, v, grid, tile)
+    sq.poll_device_error()
+    ro, ro1, rl1, rl2, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, grid, tile)
+    for a in (o, o2):
+        mx, mean = _err(_np(a), ro)
+        assert mx <= BF16_MAX and mean <= BF16_MEAN, (mx, mean)
+    assert torch.equal(inter[0], o1)  # the local pass (220-token windows) is not packed
+    assert _err(_np(lse[1]), rl2)[0] <= 2e-3
+    assert _err(_np(l2), rl2)[0] <= 2e-3
 
 
 def test_autograd_through_three_passes(cuda_ok):

@@ -84,8 +84,10 @@ struct FwdLayout {
 };
 
 // barrier indices
-enum { F_QF = 0, F_QE = 2, F_KVF = 4, F_KVE = 8, F_SF = 12, F_PF = 14, F_OF = 16, F_ST = 18, F_DRAIN = 20 };
-// (two Q slots, four key/value slots, two of the rest: one per warpgroup)
+// (two Q slots, four key/value slots, two of the rest: one per warpgroup). P is handed to
+// the tensor core in two halves of 64 keys: F_PF when the first half (and any rescale of
+// O) is in TMEM, F_PF2 when the second is.
+enum { F_QF = 0, F_QE = 2, F_KVF = 4, F_KVE = 8, F_SF = 12, F_PF = 14, F_OF = 16, F_PF2 = 18, F_DRAIN = 20 };
 
 struct Item {
   int pass, bh, pair;
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&bars[F_SF + i], 1);
       mbar_init(&bars[F_PF + i], 128);
       mbar_init(&bars[F_OF + i], 1);
-      mbar_init(&bars[F_ST + i], 128);
+      mbar_init(&bars[F_PF2 + i], 128);
     }
     mbar_init(&bars[F_DRAIN], 1);
     mbar_init(&bars[F_DRAIN + 1], 1);
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int x = warp == 9 ? 0 : 1;
     const uint32_t id_s = idesc_bf16_f32(128, 128, 0, 0);
     const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);
-    uint32_t ebase = 0, qbase = 0, pc = 0, pvc = 0;
+    uint32_t ebase = 0, qbase = 0, pc = 0;
     bool ok = true;
     for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
       const Item it = decode_item(args, i);
@@ -361,8 +363,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t ks = uk % Lay::NKV, vs = uv % Lay::NKV;
         if (!(ok = mbar_wait(&bars[F_KVF + ks], (uk / Lay::NKV) & 1, abort_flag, to))) break;
         if (k == 0 && !(ok = mbar_wait(&bars[F_QF + q % 2], (q / 2) & 1, abort_flag, to))) break;
-        // the previous P.V of this warpgroup has read P before S is overwritten
-        if (pvc > 0 && !(ok = mbar_wait(&bars[F_OF + x], (pvc - 1) & 1, abort_flag, to))) break;
+        // S overwrites the columns that the previous P.V of this warpgroup reads P from. No
+        // wait: the tensor core runs the MMAs that one thread issues in issue order, so the
+        // P.V has read its A operand before this S writes there.
         tc_fence_after();
         const uint32_t qa = sbase + Lay::Q_OFF + (q % 2) * Lay::TILE;
         const uint32_t ka = sbase + Lay::KV_OFF + ks * Lay::TILE;
@@ -377,16 +380,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_commit(&bars[F_KVE + ks]);
         if (!shared) tc_commit(&bars[F_KVE + ks]);
         if (!(ok = mbar_wait(&bars[F_PF + x], pc & 1, abort_flag, to))) break;
-        ++pc;
         if (!(ok = mbar_wait(&bars[F_KVF + vs], (uv / Lay::NKV) & 1, abort_flag, to))) break;
         tc_fence_after();
         const uint32_t va = sbase + Lay::KV_OFF + vs * Lay::TILE;
+        // keys 0-63 as soon as their P is in TMEM, keys 64-127 once the rest is
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 4; ++kk)
           mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, sdesc_sw128(va + kk * 16 * 128, kBlk, 1024), id_o,
                  (k > 0 || kk > 0) ? 1u : 0u);
+        if (!(ok = mbar_wait(&bars[F_PF2 + x], pc & 1, abort_flag, to))) break;
+        ++pc;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk)
+          mma_ts(tmem + x * 256 + 128, tmem + x * 256 + kk * 8, sdesc_sw128(va + kk * 16 * 128, kBlk, 1024), id_o, 1u);
         tc_commit(&bars[F_OF + x]);
-        ++pvc;
         tc_commit(&bars[F_KVE + vs]);
         if (!shared) tc_commit(&bars[F_KVE + vs]);
       }
@@ -522,22 +530,28 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
           tmem_st32(tS + hh * 32, pk);
-        }
-        const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
-        // the previous P.V has completed: S of this step was issued after it
-        if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (hh == 0) {
+            // O is rescaled before the first P.V half accumulates into it; the previous P.V
+            // has completed (S of this step was issued after it)
+            if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {  // two 64-column halves keep register pressure down
-            uint32_t o[64];
-            tmem_ld64(tO + h * 64, o);
+              for (int h = 0; h < 2; ++h) {  // two 64-column halves keep register pressure down
+                uint32_t o[64];
+                tmem_ld64(tO + h * 64, o);
 #pragma unroll
-            for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st64(tO + h * 64, o);
+                for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                tmem_st64(tO + h * 64, o);
+              }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[F_PF + a]);
           }
         }
+        const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&bars[F_PF + a]);
+        mbar_arrive(&bars[F_PF2 + a]);
         l_run = l_run * alpha + sum;
         m_run = m_use;
       }

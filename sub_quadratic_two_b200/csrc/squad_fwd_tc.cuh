@@ -445,7 +445,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int qt;    // query box within the problem
       int base;  // first token of the problem
       int tok;   // this thread's output row, or -1 past the box's valid rows
-      uint64_t mlo, mhi;  // packed geometry: key columns of this row's problem (bits 0-63, 64-127)
     };
     auto find_job = [&](int i) -> SJob {
       for (; i < args.total_items; i += gridDim.x) {
@@ -454,29 +453,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!J.valid) continue;
         const Geom& g = args.ps[it.pass].g;
         int tok = row < tile_valid_rows(g, J.qt) ? J.base + tile_row_offset(g, J.qt, row) : -1;
-        uint64_t mlo = ~0ull, mhi = ~0ull;
-        if (g.pk > 1) {
-          // the columns at this row's position along the packed dimension: runs of pk_rowdiv
-          // columns, one every pk * pk_rowdiv
-          const int id = pack_id(g, row), R = g.pk_rowdiv;
-          if (J.j0 + id >= g.pk_ext) tok = -1;  // past the digit's extent: zero-filled row
-          mlo = 0ull;
-          mhi = 0ull;
-          for (int s0 = id * R; s0 < 128; s0 += g.pk * R) {
-            const int e = s0 + R < 128 ? s0 + R : 128;
-            if (s0 < 64) {
-              const int e0 = e < 64 ? e : 64;
-              mlo |= (e0 - s0 >= 64 ? ~0ull : ((1ull << (e0 - s0)) - 1ull)) << s0;
-            }
-            if (e > 64) {
-              const int s1 = s0 > 64 ? s0 - 64 : 0, e1 = e - 64;
-              mhi |= (e1 - s1 >= 64 ? ~0ull : ((1ull << (e1 - s1)) - 1ull)) << s1;
-            }
-          }
-        }
-        return SJob{i, it.pass, J.qt, J.base, tok, mlo, mhi};
+        // packed geometry: a row past the packed digit's extent is a zero-filled row
+        if (g.pk > 1 && J.j0 + pack_id(g, row) >= g.pk_ext) tok = -1;
+        return SJob{i, it.pass, J.qt, J.base, tok};
       }
-      return SJob{args.total_items, 0, 0, 0, -1, ~0ull, ~0ull};
+      return SJob{args.total_items, 0, 0, 0, -1};
     };
     SJob cur = find_job(blockIdx.x);
     while (ok && cur.i < args.total_items) {
@@ -499,10 +480,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (32 * j + e >= lim) r[32 * j + e] = 0xff800000u;
           }
         }
-        if (g.pk > 1) {  // packed problems: keys of other problems in the box -> -inf
+        if (g.pk > 1) {
+          // packed problems: keys of other problems in the box -> -inf. This row's problem
+          // holds runs of pk_rowdiv columns, one run every pk * pk_rowdiv columns.
+          const int R = g.pk_rowdiv;
+          uint64_t mlo = 0ull, mhi = 0ull;
+          for (int s0 = pack_id(g, row) * R; s0 < 128; s0 += g.pk * R) {
+            const int e = s0 + R < 128 ? s0 + R : 128;
+            if (s0 < 64) {
+              const int e0 = e < 64 ? e : 64;
+              mlo |= (e0 - s0 >= 64 ? ~0ull : ((1ull << (e0 - s0)) - 1ull)) << s0;
+            }
+            if (e > 64) {
+              const int s1 = s0 > 64 ? s0 - 64 : 0, e1 = e - 64;
+              mhi |= (e1 - s1 >= 64 ? ~0ull : ((1ull << (e1 - s1)) - 1ull)) << s1;
+            }
+          }
 #pragma unroll
           for (int e = 0; e < 128; ++e)
-            if (!(((e < 64 ? cur.mlo : cur.mhi) >> (e & 63)) & 1ull)) r[e] = 0xff800000u;
+            if (!(((e < 64 ? mlo : mhi) >> (e & 63)) & 1ull)) r[e] = 0xff800000u;
         }
         // row maximum: 8 independent partial maxima of three-input max
         float mp[8];

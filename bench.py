@@ -164,12 +164,20 @@ def whole_job_throughput(world: int, flops_per_rank_step: float, ms_per_step: fl
 FWD_KERNEL_SOURCES = ("squad_fwd_tc.cuh", "sm100.cuh", "geometry.h")
 
 
+def code_only(text: str) -> str:
+    """C/C++ source with comments, trailing blanks and empty lines removed."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def source_sha(paths) -> str:
-    """First 16 hex digits of the SHA-256 of the concatenated kernel sources."""
+    """First 16 hex digits of the SHA-256 of the concatenated kernel sources, comments
+    removed (a comment edit does not change the kernel that the counters describe)."""
     h = hashlib.sha256()
     for path in paths:
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

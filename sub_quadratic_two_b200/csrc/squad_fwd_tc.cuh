@@ -20,7 +20,7 @@
 //   warps 0-3  softmax warpgroup 0, warps 4-7 softmax warpgroup 1
 //              (thread = TMEM lane = query row of the box)
 //   warp 8     TMA producer: Q boxes (two slots, a box is released after its job's
-//              last S) and key/value boxes (one ring of five slots, K and V of a key
+//              last S) and key/value boxes (one ring of four slots, K and V of a key
 //              box in consecutive slots) in the order the tensor core consumes them
 //   warps 9,11 one thread each issues tcgen05.mma for one softmax warpgroup:
 //              S = Q K^T (both operands K-major) and O += P V (P read from TMEM,
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t sbase = smem_u32(smem);
   const bool fused = args.mode == FWD_FUSED;
-  // launch: 384 x 168 registers; after: 2 x 128 x 224 (softmax) + 128 x 56 (control)
+  // 384 threads at up to 168 registers each (the launch bound); no register reallocation
 
   if (warp == 8) {
     // ================================================================ TMA producer

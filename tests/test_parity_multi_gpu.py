@@ -151,3 +151,16 @@ def test_three_passes_on_the_video_shape(cuda_ok):
         ro, _, _, _ = oracle.squad_fwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, tiles)
         mx, mean = _err(_np(o[sel]), ro)
         assert mx <= fmax and mean <= fmean, (h, mx, mean)
+
+
+def test_packed_passes_are_deterministic(cuda_ok):
+    # packed boxes (20-token windows six to a box along c, then 22-token groups five to a
+    # box along a) run the same MMAs in the same order on every call: bitwise repeatable
+    grid, tiles = (4, 22, 40), [(1, 1, 20), (2, 11, 20)]
+    inp = random_problem(59, 1, 2, 128, grid, (1, 1, 1), dtype=torch.bfloat16)
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    first = sq.squad_attn_multi_fwd(q, k, v, grid, tiles)
+    second = sq.squad_attn_multi_fwd(q, k, v, grid, tiles)
+    sq.poll_device_error()
+    for a, b in zip(first, second):
+        assert torch.equal(a, b)

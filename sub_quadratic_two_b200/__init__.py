@@ -130,6 +130,17 @@ def _check_inputs(*ts: torch.Tensor):
             raise ValueError("q, k, v (and gradients) must share shape, dtype and device")
 
 
+def _check_aux(t: torch.Tensor, shape, dtype, device, name: str):
+    """A saved tensor handed back to the library: its extent is implied by the descriptor,
+    so a wrong shape, dtype or device would make a kernel read outside it."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {dtype} of shape {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def workspace_size(desc: SquadDesc, which: int) -> int:
     out = ctypes.c_size_t(0)
     _check(load_library().squad_attn_workspace_size(ctypes.byref(desc), which, ctypes.byref(out)),
@@ -148,6 +159,11 @@ def squad_attn_fwd(q, k, v, grid, tile, scale: Optional[float] = None, save: boo
     lib = load_library()
     _check_inputs(q, k, v)
     desc = make_desc(q, grid, tile, scale)
+    if out is not None:
+        _check_aux(out, q.shape, q.dtype, q.device, "out")
+    if workspace is not None and (not workspace.is_cuda or workspace.device != q.device
+                                  or not workspace.is_contiguous()):
+        raise ValueError(f"workspace must be a contiguous CUDA tensor on {q.device}")
     o = torch.empty_like(q) if out is None else out
     if save:
         o1 = torch.empty_like(q)
@@ -175,6 +191,8 @@ def squad_attn_fwd_pass(stage: int, q, k, val, out, grid, tile, scale: Optional[
     """One pass of the forward (stage 1: local, values V; stage 2: global, values O1) into ``out``."""
     lib = load_library()
     _check_inputs(q, k, val, out)
+    if lse is not None:
+        _check_aux(lse, q.shape[:3], torch.float32, q.device, "lse")
     desc = make_desc(q, grid, tile, scale)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -196,6 +214,8 @@ def squad_attn_bwd(q, k, v, o, o1, lse1, lse2, dout, grid, tile, scale: Optional
     """Backward through the C ABI. Returns (dq, dk, dv)."""
     lib = load_library()
     _check_inputs(q, k, v, o, o1, dout)
+    for t, name in ((lse1, "lse1"), (lse2, "lse2")):
+        _check_aux(t, q.shape[:3], torch.float32, q.device, name)
     desc = make_desc(q, grid, tile, scale)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws_bytes = workspace_size(desc, 1)
@@ -203,7 +223,7 @@ def squad_attn_bwd(q, k, v, o, o1, lse1, lse2, dout, grid, tile, scale: Optional
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
         _check(lib.squad_attn_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o1),
-                                  _ptr(lse1.contiguous()), _ptr(lse2.contiguous()), _ptr(dout), _ptr(dq), _ptr(dk),
+                                  _ptr(lse1), _ptr(lse2), _ptr(dout), _ptr(dq), _ptr(dk),
                                   _ptr(dv), _ptr(ws), ws_bytes, st), "squad_attn_bwd")
     return dq, dk, dv
 
@@ -267,6 +287,11 @@ def squad_attn_fwd_noalloc(q, k, v, grid, tile, scale: Optional[float] = None, o
     fn.restype = ctypes.c_int
     _check_inputs(q, k, v)
     desc = make_desc(q, grid, tile, scale)
+    if out is not None:
+        _check_aux(out, q.shape, q.dtype, q.device, "out")
+    for t, name in ((lse1, "lse1"), (lse2, "lse2")):
+        if t is not None:
+            _check_aux(t, q.shape[:3], torch.float32, q.device, name)
     o = torch.empty_like(q) if out is None else out
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
@@ -312,6 +337,8 @@ def squad_attn_multi_bwd(q, k, v, o, inter, lse, dout, grid, tiles, scale: Optio
     _check_inputs(q, k, v, o, dout)
     desc = make_desc(q, grid, tiles[0], scale)
     nt, tarr = _tiles_arg(tiles)
+    _check_aux(inter, (nt,) + tuple(q.shape), q.dtype, q.device, "inter")
+    _check_aux(lse, (nt + 1,) + tuple(q.shape[:3]), torch.float32, q.device, "lse")
     ws_bytes = ctypes.c_size_t(0)
     _check(lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(desc), nt, tarr, ctypes.byref(ws_bytes)),
            "squad_attn_multi_bwd_workspace_size")
@@ -320,7 +347,7 @@ def squad_attn_multi_bwd(q, k, v, o, inter, lse, dout, grid, tiles, scale: Optio
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
         _check(lib.squad_attn_multi_bwd(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                        _ptr(inter.contiguous()), _ptr(lse.contiguous()), _ptr(dout), _ptr(dq),
+                                        _ptr(inter), _ptr(lse), _ptr(dout), _ptr(dq),
                                         _ptr(dk), _ptr(dv), _ptr(ws), int(ws_bytes.value), st),
                "squad_attn_multi_bwd")
     return dq, dk, dv

@@ -149,3 +149,36 @@ def test_tiles_that_do_not_nest_are_rejected():
     for tiles in ([(1, 3, 1)], [(1, 2, 4), (1, 4, 2)], [(2, 2, 2), (1, 1, 1)]):
         with pytest.raises(ValueError):
             oracle.squad_fwd_multi(q, k, v, (2, 4, 8), tiles)
+
+
+@pytest.mark.parametrize("grid,tiles", [
+    ((2, 4, 6), [(1, 2, 3)]),
+    ((2, 4, 8), [(1, 1, 2), (1, 2, 4)]),
+    ((4, 4, 4), [(1, 1, 2), (2, 2, 2), (2, 4, 4)]),
+])
+def test_uniform_scores_give_the_mean_of_v(grid, tiles):
+    # With Q = 0 every score is 0 and every softmax is uniform over its group. Pass 1
+    # then gives each token the mean of V over its t_1-window; pass j averages those
+    # window means over the t_{j-1}-windows inside a t_j-window, i.e. the mean of V over
+    # the t_j-window; the last pass gives the mean of V over the whole grid, for every
+    # token. Each LSE is log of the pass's group size.
+    q, k, v, _ = _problem(11, grid, d=8)
+    q = torch.zeros_like(q)
+    o, inter, lse, _ = oracle.squad_fwd_multi(q, k, v, grid, tiles)
+    vn = v.numpy()
+    want = np.broadcast_to(vn.mean(axis=2, keepdims=True), vn.shape)
+    np.testing.assert_allclose(o, want, rtol=0, atol=1e-12)
+    # intermediate j: mean of V over the token's t_j-window
+    T, H, W = grid
+    t, y, x = _coords(grid)
+    for j, tile in enumerate(tiles):
+        win = ((t // tile[0]) * (H // tile[1]) + y // tile[1]) * (W // tile[2]) + x // tile[2]
+        exp = np.zeros_like(vn)
+        for wdx in np.unique(win):
+            sel = win == wdx
+            exp[:, :, sel, :] = vn[:, :, sel, :].mean(axis=2, keepdims=True)
+        np.testing.assert_allclose(inter[j], exp, rtol=0, atol=1e-12)
+    chain = [(1, 1, 1)] + [tuple(tl) for tl in tiles] + [tuple(grid)]
+    for j, (inner, outer) in enumerate(zip(chain[:-1], chain[1:])):
+        size = np.prod(outer) // np.prod(inner)
+        np.testing.assert_allclose(lse[j], np.log(size), rtol=0, atol=1e-12)

@@ -135,6 +135,20 @@ int main() {
       if (seen[t] != 1) return fail("pack coverage", it, t, seen[t]);
   }
   if (packed_geoms < 50) return fail("too few packed geometries", packed_geoms, 0, 0);
+  // the three passes over the 27,280-token grid used by the benchmark: 20-token windows six
+  // to a box along c (four groups per window column), 11-token groups ten to a box along
+  // c, 124-token groups unpacked
+  {
+    Geom g1 = make_geom_pass(1, 24, 31, 22, 40, 1, 1, 1, 1, 1, 20);
+    if (!plan_pack(g1) || g1.pk != 6 || g1.pk_dim != 2 || g1.pk_ext != 22 || g1.probs != 2 * 4 * 31)
+      return fail("video pass 1 packing", g1.pk, g1.pk_dim, g1.probs);
+    Geom g2 = make_geom_pass(1, 24, 31, 22, 40, 1, 1, 20, 1, 11, 20);
+    if (!plan_pack(g2) || g2.pk != 10 || g2.pk_dim != 2 || g2.pk_ext != 20 || g2.probs != 2 * 2 * 2 * 31)
+      return fail("video pass 2 packing", g2.pk, g2.pk_dim, g2.probs);
+    Geom g3 = make_geom_pass(1, 24, 31, 22, 40, 1, 11, 20, 31, 22, 40);
+    if (plan_pack(g3) || g3.pk != 1) return fail("video pass 3 packing", g3.pk, g3.L, 0);
+    checked += 3;
+  }
   std::printf("ok %lld\n", checked);
   return 0;
 }

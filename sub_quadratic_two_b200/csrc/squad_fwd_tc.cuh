@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     while (ok && cur.i < args.total_items) {
       const PassArgs& P = args.ps[cur.pass];
       const Geom& g = P.g;
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
       for (int k = 0; k < g.nt; ++k) {
         if (!(ok = wwait(&bars[F_SF + a], sc & 1))) break;
         ++sc;
@@ -511,25 +511,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
         // exact running maximum: the largest P of a row is exactly 1 before its bf16
         // rounding, which keeps the dominant term of peaked rows exact
-        const float m_use = fmaxf(m_run, mx);
-        const float alpha = ex2_approx((m_run - m_use) * c2);
+        // the first key box sets the maximum; a later one moves it only when it grows by more
+        // than 2^8 (then O and the sums are rescaled), else its probabilities may exceed 1
+        float m_use = mx, alpha = 1.f;
+        bool grow = false;
+        if (k > 0) {
+          grow = (mx - m_run) * c2 > 8.f;
+          m_use = grow ? mx : m_run;
+          alpha = grow ? ex2_approx((m_run - mx) * c2) : 1.f;
+        }
         const float neg = -m_use * c2;
-        float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint64_t c2x2 = f2(c2, c2), negx2 = f2(neg, neg);
+        uint64_t sl[2] = {0ull, 0ull};  // paired partial sums of p
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // two 64-column halves: P of a half is packed and stored at once
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 64; e += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(r[64 * hh + e]), c2, neg));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(r[64 * hh + e + 1]), c2, neg));
-            sp[(e >> 1) & 7] += p0 + p1;
+            const uint64_t x2 = ffma2(f2(__uint_as_float(r[64 * hh + e]), __uint_as_float(r[64 * hh + e + 1])),
+                                      c2x2, negx2);
+            const float p0 = ex2_approx(f2_lo(x2));
+            const float p1 = ex2_approx(f2_hi(x2));
+            sl[(e >> 1) & 1] = fadd2(sl[(e >> 1) & 1], f2(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
           tmem_st32(tS + hh * 32, pk);
           if (hh == 0) {
             // O is rescaled before the first P.V half accumulates into it; the previous P.V
             // has completed (S of this step was issued after it)
-            if (k > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
               for (int h = 0; h < 2; ++h) {  // two 64-column halves keep register pressure down
                 uint32_t o[64];
@@ -544,11 +554,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_arrive(&bars[F_PF + a]);
           }
         }
-        const float sum = ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        const uint64_t s2 = fadd2(sl[0], sl[1]);
+        const float sum = f2_lo(s2) + f2_hi(s2);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&bars[F_PF2 + a]);
+        // the box's largest probability enters the normalising sum rounded to bf16, as the
+        // tensor core sees it, so that a row dominated by one key returns its value exactly
+        const float pmax = ex2_approx(fmaf(mx, c2, neg));
+        const float pmax_bf = __uint_as_float(pack_bf16x2(0.f, pmax) & 0xffff0000u);
         l_run = l_run * alpha + sum;
+        lr_run = lr_run * alpha + (pmax_bf - pmax);
         m_run = m_use;
       }
       if (!ok) break;
@@ -562,7 +578,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       {
         // Each thread holds its own row. A warp passes its 32 rows through a private
         // 128B-swizzled patch so that every global store writes four whole 128-byte lines.
-        const float inv = 1.f / l_run;
+        const float inv = 1.f / (l_run + lr_run);
         const uint32_t xp = sbase + Lay::XP_OFF + (warp & 7) * 4096;
         const int lr = lane >> 3, lc = lane & 7;  // read-back: row 4*i + lr, 16-byte chunk lc
         int rtok[8];

@@ -6,7 +6,9 @@ passes, each of which rounds its probabilities to bf16 before the P.V product an
 stores its output in bf16; a pass passes the error of its values on through a
 convex combination, so the errors of k passes add. The bf16 bounds here are
 therefore the two-pass ones times k / 2 (three passes: max 2.25e-2, mean 3e-3;
-gradients 4.5e-2). Reading of the
+gradients 4.5e-2). tests/test_kpass_error_budget.py pins this budget on the CPU with a
+model of the two roundings per pass (additivity over passes; three passes on the
+27,280-token shape reach about 2e-2 from rounding alone). Reading of the
 pages' outlook on composing more than two passes ("SQuad: Sub-Quadratic
 Attention Distillation for Efficient Video Generation", gist.science technical
 summary, Significance and Claims): nested tiles, pass j attends within a

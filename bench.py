@@ -202,6 +202,18 @@ def cpu_cores():
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first "model name" line of /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def oracle_sample(wl, budget_s: float, threads: int):
     """The fp64 oracle, as it stands, over whole heads of the workload until the budget is spent."""
     import oracle
@@ -251,7 +263,8 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "sample": "1 of %d heads" % wl.heads, "grid": list(wl.grid),
                    "tile": list(wl.tile), "d": wl.d},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "threads": cores, "kind": "oracle",
+                         "sample": sample, "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -512,8 +525,12 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = cpu_cores()
         fl, secs, heads = oracle_sample(wl, args.cpu_seconds, cores)
-        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{heads} of {wl.heads} heads of {wl.name} (fp64, {secs:.1f} s)"}
+        fl1, secs1, heads1 = oracle_sample(wl, args.cpu_seconds / 2, 1)
+        cpu = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": cores, "threads": cores, "kind": "oracle",
+               "sample": f"{heads} of {wl.heads} heads of {wl.name} (fp64, {secs:.1f} s)",
+               "cpu_model": cpu_model(),
+               "single_core": {"value": fl1 / secs1 / 1e12, "unit": "TFLOP/s", "threads": 1,
+                               "sample": f"{heads1} of {wl.heads} heads of {wl.name} (fp64, {secs1:.1f} s)"}}
 
     if rank == 0:
         line = {

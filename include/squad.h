@@ -121,8 +121,10 @@ squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* 
  *     contents. Each call overwrites every element it later reads, so nothing
  *     needs clearing, but calls whose kernels overlap on the GPU (different
  *     streams, or different host threads) race on the array: serialise them.
- *   - Arguments and results are those of squad_attn_fwd with o1 == NULL;
- *     lse1 and lse2 may be NULL. */
+ *   - Arguments are those of squad_attn_fwd with o1 == NULL; lse1 and lse2 may
+ *     be NULL. The two passes run as two launches (squad_attn_fwd fuses them
+ *     into one); each row is computed by the same kernel code, and the results
+ *     agree with squad_attn_fwd's within the tolerances its tests state. */
 #define SQUAD_NOALLOC_SCRATCH_BYTES (32u << 20)
 squad_status squad_attn_fwd_noalloc(const squad_desc* desc, const void* q, const void* k, const void* v,
                                     void* o, float* lse1, float* lse2, void* stream);
@@ -212,6 +214,14 @@ const char* squad_strerror(int status);
 
 /* cudaError_t / CUresult value of the last failing CUDA call on this thread. */
 int squad_last_cuda_error(void);
+
+/* Counters of the library's tensor-map cache (no counterpart in the paper). Every
+ * call that launches a tensor-core kernel needs TMA tensor maps (eight per forward
+ * launch, four per backward pass); their encoding is a host driver call, and maps
+ * already made for the same device, pointers and shapes are reused instead: hits
+ * counts the reused ones, misses the encoded ones, since the library was loaded and
+ * over all threads. Either pointer may be NULL (not both). No CUDA call is made. */
+squad_status squad_tmap_cache_stats(unsigned long long* hits, unsigned long long* misses);
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int squad_version(void);

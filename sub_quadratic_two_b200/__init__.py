@@ -23,6 +23,7 @@ __all__ = [
     "SquadError", "attention", "squad_attn_fwd", "squad_attn_bwd", "workspace_size",
     "poll_device_error", "library_path", "load_library", "SQUAD_F32", "SQUAD_BF16", "squad_attn_fwd_pass",
     "plan_info", "make_desc", "attention_multi", "squad_attn_multi_fwd", "squad_attn_multi_bwd",
+    "tmap_cache_stats",
 ]
 
 SQUAD_F32 = 0
@@ -75,12 +76,14 @@ def load_library():
         lib.squad_attn_multi_bwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp,
                                              sz, vp]
         lib.squad_poll_device_error.argtypes = [vp]
+        ull = ctypes.POINTER(ctypes.c_ulonglong)
+        lib.squad_tmap_cache_stats.argtypes = [ull, ull]
         lib.squad_strerror.argtypes = [ctypes.c_int]
         lib.squad_strerror.restype = ctypes.c_char_p
         for f in ("squad_attn_workspace_size", "squad_attn_fwd", "squad_attn_bwd", "squad_poll_device_error",
                   "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_multi_fwd",
                   "squad_attn_multi_bwd_workspace_size", "squad_attn_multi_bwd",
-                  "squad_last_cuda_error", "squad_version"):
+                  "squad_last_cuda_error", "squad_version", "squad_tmap_cache_stats"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -235,6 +238,13 @@ def selftest_wait_timeout(timeout_ns: int = 10_000_000, stream: Optional[torch.c
     lib.squad_selftest_wait_timeout.restype = ctypes.c_int
     dev = torch.device("cuda", torch.cuda.current_device())
     _check(lib.squad_selftest_wait_timeout(int(timeout_ns), _stream_handle(stream, dev)), "squad_selftest_wait_timeout")
+
+
+def tmap_cache_stats() -> Tuple[int, int]:
+    """(hits, misses) of the library's tensor-map cache since it was loaded."""
+    hits, misses = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+    _check(load_library().squad_tmap_cache_stats(ctypes.byref(hits), ctypes.byref(misses)), "squad_tmap_cache_stats")
+    return int(hits.value), int(misses.value)
 
 
 def poll_device_error(stream: Optional[torch.cuda.Stream] = None, device=None):

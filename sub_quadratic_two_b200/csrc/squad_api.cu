@@ -17,6 +17,7 @@
 #include "squad_bwd_fused.cuh"
 #include "squad_fwd_tc.cuh"
 #include "squad_simt.cuh"
+#include "tmap_cache.h"
 
 namespace {
 
@@ -155,6 +156,9 @@ BwdWs bwd_workspace(const Plan& p, const squad_desc* d) {
 
 // 5-D map over a [rows, d] bf16 tensor: (d, a, b, c, token) with the problem box's
 // token strides; boxes of (64, a_n, b_sub, c_sub, 1), 128-byte swizzle.
+// Encoded maps are reused by later calls with the same pointers and shapes (tmap_cache.h).
+sq::TmapCache<128> g_tmaps;
+
 squad_status encode_map(CUtensorMap* m, const void* base, const Geom& g, int d, long long rows) {
   const cuuint64_t esz = 2;
   // a packed dimension spans the packed digit's full extent (its rows past that extent read as zeros)
@@ -165,9 +169,15 @@ squad_status encode_map(CUtensorMap* m, const void* base, const Geom& g, int d, 
                            cuuint64_t(d) * esz};
   cuuint32_t box[5] = {64u, cuuint32_t(g.a_n), cuuint32_t(g.b_sub), cuuint32_t(g.c_sub), 1u};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  int dev = 0;
+  SQ_CUDA(cudaGetDevice(&dev));
+  const sq::TmapKey key = sq::make_tmap_key(dev, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_128B, 5, base,
+                                            dims, strides, box);
+  CUresult r = g_tmaps.get(key, m, [&](CUtensorMap* out) {
+    return g_encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  });
   if (r != CUDA_SUCCESS) return cuda_fail(int(r));
   return SQUAD_OK;
 }
@@ -675,6 +685,12 @@ const char* squad_strerror(int status) {
 }
 
 int squad_last_cuda_error(void) { return t_last_cuda; }
+
+squad_status squad_tmap_cache_stats(unsigned long long* hits, unsigned long long* misses) {
+  if (hits == nullptr && misses == nullptr) return SQUAD_ERR_INVALID_ARG;
+  g_tmaps.stats(hits, misses);
+  return SQUAD_OK;
+}
 
 int squad_version(void) { return kVersion; }
 

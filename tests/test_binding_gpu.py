@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import sub_quadratic_two_b200 as sq
-from workloads import random_problem
+from workloads import WORKLOADS, make_inputs, random_problem
 
 pytestmark = pytest.mark.gpu
 
@@ -48,3 +48,25 @@ def test_forward_rejects_mismatched_outputs(cuda_ok):
     with pytest.raises(ValueError):
         sq.squad_attn_fwd_noalloc(q, k, v, grid, tile, lse1=torch.empty(3, device=q.device, dtype=torch.float32))
     sq.poll_device_error()
+
+
+def test_repeated_call_reuses_its_tensor_maps(cuda_ok):
+    # a forward launch needs eight TMA tensor maps; a second call with the same pointers
+    # and shapes takes all eight from the library's cache and encodes none
+    wl = WORKLOADS["small_bf16"]
+    inp = make_inputs(wl)
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    ws = torch.empty(sq.workspace_size(sq.make_desc(q, wl.grid, wl.tile, None), 0), device="cuda", dtype=torch.uint8)
+    sq.squad_attn_fwd(q, k, v, wl.grid, wl.tile, save=False, out=o, workspace=ws)
+    hits0, misses0 = sq.tmap_cache_stats()
+    sq.squad_attn_fwd(q, k, v, wl.grid, wl.tile, save=False, out=o, workspace=ws)
+    hits1, misses1 = sq.tmap_cache_stats()
+    sq.poll_device_error()
+    assert misses1 == misses0 and hits1 == hits0 + 8
+    o2 = torch.empty_like(q)   # another output buffer: only its map is new
+    sq.squad_attn_fwd(q, k, v, wl.grid, wl.tile, save=False, out=o2, workspace=ws)
+    hits2, misses2 = sq.tmap_cache_stats()
+    sq.poll_device_error()
+    assert misses2 == misses1 + 1 and hits2 == hits1 + 7
+    assert torch.equal(o, o2)

@@ -113,3 +113,30 @@ def test_k_pass_writes_stay_inside_their_buffers(cuda_ok, grid, tiles, dtype):
     sq.poll_device_error()
     for name, g in (("o", o), ("inter", inter), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("ws", ws)):
         assert g.intact(), name
+
+
+@pytest.mark.parametrize("grid,tile,heads,d", [
+    ((4, 22, 40), (1, 11, 20), 2, 128),   # 220-token windows: ragged boxes 120 + 100
+    ((2, 10, 88), (1, 5, 88), 1, 128),    # 440-token windows in five boxes
+    ((8, 16, 16), (2, 4, 8), 3, 64),      # d = 64, tT > 1
+])
+def test_inference_forward_writes_stay_inside_their_buffers(cuda_ok, grid, tile, heads, d):
+    # o1 == NULL: the local-pass output and the per-head counters live in the workspace
+    # (squad_attn_workspace_size(desc, 0)), and consumed local-pass rows are dropped from
+    # L2 after the global pass reads them
+    lib = sq.load_library()
+    inp = random_problem(75, 1, heads, d, grid, tile, dtype=torch.bfloat16)
+    dev = torch.device("cuda", 0)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    desc = sq.make_desc(q, grid, tile, None)
+    o = Guarded(q.shape, q.dtype, dev)
+    need = sq.workspace_size(desc, 0)
+    ws = Guarded((need,), torch.uint8, dev)
+    assert lib.squad_attn_fwd(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), None, None, None, _p(ws), need,
+                              _stream()) == 0
+    torch.cuda.synchronize()
+    sq.poll_device_error()
+    assert o.intact() and ws.intact()
+    ref, *_ = sq.squad_attn_fwd(q, k, v, grid, tile, save=True)
+    sq.poll_device_error()
+    assert torch.equal(o.t, ref)

@@ -158,6 +158,23 @@ def test_long_video_forward_full_size(cuda_ok):
     check_fwd_bf16(inp, wl.grid, wl.tile, heads=[7])
 
 
+@pytest.mark.parametrize("name,heads", [("wan5b_fwd", [0, 13, 23]), ("long_video", [7])])
+def test_inference_forward_full_size(cuda_ok, name, heads):
+    # the path the benchmark times: no saved outputs, the local-pass output in the workspace
+    # and each consumed row of it dropped from L2 after its single read; whole heads are
+    # compared with the oracle
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    qd, kd, vd = _dev(inp.q, inp.k, inp.v)
+    o, o1, l1, l2 = sq.squad_attn_fwd(qd, kd, vd, wl.grid, wl.tile, save=False)
+    sq.poll_device_error()
+    assert o1 is None and l1 is None and l2 is None
+    o = o.cpu().double().numpy()
+    sel = (slice(0, 1), heads)
+    ro, _, _, _, _ = oracle.squad_fwd(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, wl.tile)
+    assert_bf16_fwd(o[sel], ro, "O")
+
+
 # ------------------------------------------------------------------ bf16 backward
 
 @pytest.mark.parametrize("grid,tile,heads,d", [

@@ -95,3 +95,72 @@ def test_noalloc_python_binding(cuda_ok):
     got = sq.squad_attn_fwd_noalloc(q, k, v, wl.grid, wl.tile)
     sq.poll_device_error()
     _close(got, ref, False, "O")
+
+
+def test_noalloc_matches_the_oracle(cuda_ok):
+    # all eight heads of the small bf16 workload against the fp64 oracle directly
+    import oracle
+    fn = _abi()
+    wl, inp = _inputs("small_bf16", False)
+    q, k, v = (t.cuda().contiguous() for t in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    l1, l2 = (torch.empty(q.shape[:3], device=q.device) for _ in range(2))
+    desc = sq.make_desc(q, wl.grid, wl.tile, None)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert fn(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), _p(l1), _p(l2), stream) == 0
+    sq.poll_device_error()
+    ro, _, rl1, rl2, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, wl.grid, wl.tile)
+    _close(o.cpu(), torch.from_numpy(ro), False, "O")
+    assert (l1.cpu().double() - torch.from_numpy(rl1)).abs().max().item() <= LSE_TOL
+    assert (l2.cpu().double() - torch.from_numpy(rl2)).abs().max().item() <= LSE_TOL
+
+
+def test_noalloc_at_the_exact_scratch_size(cuda_ok):
+    # bf16 [1, 8, 16384, 128]: the local-pass output is exactly 32 MiB, every byte of the
+    # scratch array is written and read; compared with squad_attn_fwd (the same kernels,
+    # one fused launch) and, on one head, with the oracle
+    import oracle
+    from workloads import random_problem as rp
+    fn = _abi()
+    grid, tile = (16, 32, 32), (1, 8, 16)
+    inp = rp(99, 1, 8, 128, grid, tile, dtype=torch.bfloat16)
+    assert 1 * 8 * 16384 * 128 * 2 == SCRATCH_BYTES
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    o = torch.empty_like(q)
+    desc = sq.make_desc(q, grid, tile, None)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        assert fn(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o), None, None, stream) == 0
+    ref, *_ = sq.squad_attn_fwd(q, k, v, grid, tile, save=False)
+    sq.poll_device_error()
+    _close(o, ref, False, "O vs squad_attn_fwd")
+    ro, *_ = oracle.squad_fwd(inp.q[:, 5:6], inp.k[:, 5:6], inp.v[:, 5:6], grid, tile)
+    _close(o[:, 5:6].cpu(), torch.from_numpy(ro), False, "O vs oracle")
+
+
+def test_noalloc_rejects_one_row_past_the_scratch(cuda_ok):
+    fn = _abi()
+    fake = ctypes.c_void_p(0x10000)   # never touched: the size check comes first
+    # fp32 [1, 1, 262144, 32] is exactly 32 MiB: accepted up to the size check; 262145
+    # tokens (grid 5 x 13 x 4033) is one 128-byte row more: rejected before any launch
+    over = sq.SquadDesc(1, 1, 32, 5, 13, 4033, 1, 1, 1, sq.SQUAD_F32, 0.0)
+    assert 262145 * 32 * 4 == SCRATCH_BYTES + 128
+    assert fn(ctypes.byref(over), fake, fake, fake, fake, None, None, None) == 7   # SQUAD_ERR_WORKSPACE
+
+
+def test_noalloc_writes_stay_inside_their_buffers(cuda_ok):
+    # guard bands around o, lse1 and lse2 (the only memory the call writes besides its
+    # internal scratch): both ends keep their pattern
+    from test_guard_bands_gpu import Guarded
+    fn = _abi()
+    for name in ("small_bf16", "tiny_fp32"):
+        wl, inp = _inputs(name, False)
+        q, k, v = (t.cuda().contiguous() for t in (inp.q, inp.k, inp.v))
+        o = Guarded(q.shape, q.dtype, q.device)
+        l1, l2 = (Guarded(q.shape[:3], torch.float32, q.device) for _ in range(2))
+        desc = sq.make_desc(q, wl.grid, wl.tile, None)
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        assert fn(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(o.t), _p(l1.t), _p(l2.t), stream) == 0
+        torch.cuda.synchronize()
+        sq.poll_device_error()
+        assert o.intact() and l1.intact() and l2.intact(), name

@@ -50,6 +50,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", choices=["replicas", "sp"], default="replicas",
+                    help="replicas: every rank runs the whole workload (independent problems, weak scaling); "
+                         "sp: the workload's frames are sharded over the ranks and the two passes exchange rows "
+                         "with NCCL all-to-alls (strong scaling)")
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -271,12 +275,94 @@ def run_reference(args):
     return 0
 
 
+# ------------------------------------------------------------------ sequence-parallel arm
+
+def run_sp(args):
+    """Strong scaling: one workload, its frames sharded over the ranks (sub_quadratic_two_b200.sp)."""
+    import socket
+
+    import torch
+    import torch.distributed as dist
+
+    import sub_quadratic_two_b200 as sq
+    from sub_quadratic_two_b200.sp import SpPlan, sp_attention_fwd
+    from workloads import WORKLOADS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world == 1 and "MASTER_PORT" not in os.environ:
+        with socket.socket() as s_:
+            s_.bind(("127.0.0.1", 0))
+            os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(s_.getsockname()[1]), RANK="0",
+                              WORLD_SIZE="1")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    peaks, peak_src = load_peaks()
+    wl = WORKLOADS[args.workload]
+    plan = SpPlan(wl.B, wl.heads, wl.d, wl.grid, wl.tile, world, rank)
+    inp = make_inputs(wl)
+    H, W = wl.grid[1], wl.grid[2]
+    lo, hi = plan.t0 * H * W, (plan.t0 + plan.T) * H * W
+    q, k, v = (t[:, :, lo:hi].contiguous().to(dev) for t in (inp.q, inp.k, inp.v))
+    del inp
+    flush = torch.empty(L2_FLUSH_BYTES, device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(max(3, args.warmup)):
+        sp_attention_fwd(q, k, v, plan)
+    sq.poll_device_error()
+    sampler = ClockSampler(local)
+    sampler.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        dist.barrier()
+        starts[i].record(stream)
+        sp_attention_fwd(q, k, v, plan)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.perf_counter()
+    dist.barrier()
+    sampler.stop()
+    sq.poll_device_error()
+    ms = max_over_ranks(sum(s_.elapsed_time(e) for s_, e in zip(starts, ends)), dev) / args.steps
+    flops = wl.fwd_flops()
+    value = flops / (ms / 1e3) / 1e12
+    if rank == 0:
+        rows = plan.B * plan.heads
+        xbytes = 2 * (3 + 1) * rows * wl.n * wl.d * (world - 1) / world   # Q, K, O1 out and O back, off-rank share
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
+                       "grid": list(wl.grid), "tile": list(wl.tile), "useful_flops_per_step": flops,
+                       "l2": "flushed (512 MiB write) before every timed step",
+                       "parallelism": f"sequence-parallel x{world} (frames sharded; two NCCL all-to-alls per step)"},
+            "exchange_bytes_per_step_all_ranks": xbytes,
+            "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"], "source": peak_src},
+            "roofline": None, "cpu_baseline": None, "e2e": None,
+            "gpu_launches": args.steps * 8, "clocks": sampler.summary(t_wall0, t_wall1),
+            "note": "each step: local pass, pack, all-to-all, unpack, global pass, pack, all-to-all, unpack",
+        }
+        print(json.dumps(line))
+    dist.destroy_process_group()
+    return 0
+
+
 # ------------------------------------------------------------------ our arm
 
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode == "sp":
+        return run_sp(args)
 
     import torch
     import torch.distributed as dist

@@ -45,7 +45,8 @@ typedef enum {
   SQUAD_ERR_UNSUPPORTED = 4,  /* valid operator, but outside what the kernels handle (see below) */
   SQUAD_ERR_CUDA = 5,         /* a CUDA runtime or driver call failed (see squad_last_cuda_error) */
   SQUAD_ERR_TIMEOUT = 6,      /* a kernel gave up on a bounded wait (see squad_poll_device_error) */
-  SQUAD_ERR_WORKSPACE = 7     /* workspace missing or smaller than squad_attn_workspace_size */
+  SQUAD_ERR_WORKSPACE = 7,    /* workspace missing or smaller than squad_attn_workspace_size */
+  SQUAD_ERR_INDEX = 8         /* a shuffle kernel met a row index out of range (squad_poll_device_error) */
 } squad_status;
 
 typedef enum { SQUAD_F32 = 0, SQUAD_BF16 = 1 } squad_dtype;
@@ -188,6 +189,58 @@ squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int*
                                   const void* dout, void* dq, void* dk, void* dv, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* ---- Sequence-parallel forward over G ranks ----
+ * Sharded by windows, the local pass needs nothing from other ranks, and the
+ * global pass needs one row of every window for each in-window position (the
+ * operator of "SQuad: Sub-Quadratic Attention Distillation for Efficient Video
+ * Generation", gist.science technical summary, Methodology section 1). Rank r
+ * holds the tokens of a contiguous range of whole tT-frame windows (frames
+ * split as evenly as the frame windows allow) and, for the global pass, a range
+ * of in-window positions (split as evenly as possible). The forward on each rank:
+ *   1. local pass on its shard (squad_attn_fwd_pass, stage 1, grid T_r x H x W);
+ *   2. squad_sp_pack of Q, K and the local-pass output with map send1;
+ *   3. all-to-all (the caller's collective, e.g. NCCL) with counts send1/recv1;
+ *   4. squad_sp_unpack with maps recv1_src/recv1_row into the position-major
+ *      layout [position][window], which is the grid (P_r*T/tT) x (H/tH) x (W/tW)
+ *      with tile (T/tT) x (H/tH) x (W/tW): each of its windows is one global-pass
+ *      group, so
+ *   5. the global pass is squad_attn_fwd_pass stage 1 on that grid;
+ *   6. squad_sp_pack of its output with map send2, all-to-all with counts
+ *      send2/recv2, squad_sp_unpack with recv2_src/recv2_row: the output rows
+ *      back in the shard's token order.
+ * No counterpart in the pages beyond the operator itself; the exchange is the
+ * plainest one the two passes allow. desc describes the whole problem; G ranks
+ * (1..64, at most the number of frame windows and of positions). */
+
+/* info[8]: [0] first frame of rank `rank`, [1] its frames, [2] its tokens n_local
+ * (= frames*H*W), [3] its position-major rows n_pos (= positions*m), [4] its
+ * first position, [5] its positions, [6] w, [7] m. Host only. */
+squad_status squad_sp_plan_info(const squad_desc* desc, int G, int rank, int* info);
+
+/* The index maps of rank `rank` (host arrays, in rows of one (batch, head) slice):
+ * counts[4*G] = rows per peer of send1, recv1, send2, recv2 (in that order);
+ * send1[n_local], recv1_src[n_pos], recv1_row[n_pos], send2[n_pos],
+ * recv2_src[n_local], recv2_row[n_local] (meaning as in the steps above). Host only. */
+squad_status squad_sp_plan_maps(const squad_desc* desc, int G, int rank, int* counts, int* send1, int* recv1_src,
+                                int* recv1_row, int* send2, int* recv2_src, int* recv2_row);
+
+/* Pack rows for an all-to-all: dst holds, peer after peer, [tensor][slice][counts[q]]
+ * rows; row i of peer q, tensor t, slice s is row idx[prefix_q + i] of slice s of
+ * srcs[t] (srcs: ntensors <= 3 device tensors [slices, rows_in, row_bytes]).
+ * counts: host [G]; idx: device int32 [sum counts]; row_bytes a multiple of 16.
+ * An index outside [0, rows_in) skips that row and sets the device error word. */
+squad_status squad_sp_pack(const void* const* srcs, int ntensors, int slices, int rows_in, int row_bytes, int G,
+                           const int* counts, const int* idx, void* dst, void* stream);
+
+/* Unpack rows received from an all-to-all (src laid out as squad_sp_pack writes, with
+ * counts[q] rows per slice from peer q): row j of slice s of dsts[t] is row src_row[j]
+ * of peer src_rank[j]'s block for tensor t, slice s. dsts: ntensors device tensors
+ * [slices, rows_out, row_bytes]; src_rank, src_row: device int32 [rows_out]. An out
+ * of range peer or row skips that row and sets the device error word. */
+squad_status squad_sp_unpack(const void* src, int ntensors, int slices, int rows_out, int row_bytes, int G,
+                             const int* counts, const int* src_rank, const int* src_row, void* const* dsts,
+                             void* stream);
+
 /* Geometry the kernels use for one pass (stage 1 = local/window pass,
  * stage 2 = global/cross-window pass), for tests and byte accounting.
  * Writes 8 ints to info: [0] rows per problem (w or m), [1] problems per
@@ -206,7 +259,8 @@ squad_status squad_selftest_wait_timeout(unsigned long long timeout_ns, void* st
 
 /* Synchronises `stream`, then reads and clears the library's device error
  * word. Returns SQUAD_ERR_TIMEOUT if a kernel gave up on a bounded wait since
- * the last poll, SQUAD_ERR_CUDA if the synchronisation failed, else SQUAD_OK. */
+ * the last poll, SQUAD_ERR_INDEX if a shuffle kernel skipped a row whose index
+ * was out of range, SQUAD_ERR_CUDA if the synchronisation failed, else SQUAD_OK. */
 squad_status squad_poll_device_error(void* stream);
 
 /* Human-readable name of a status code (static storage). */

@@ -29,7 +29,8 @@ __all__ = [
 SQUAD_F32 = 0
 SQUAD_BF16 = 1
 _STATUS = {0: "SQUAD_OK", 1: "SQUAD_ERR_INVALID_ARG", 2: "SQUAD_ERR_SHAPE", 3: "SQUAD_ERR_ALIGN",
-           4: "SQUAD_ERR_UNSUPPORTED", 5: "SQUAD_ERR_CUDA", 6: "SQUAD_ERR_TIMEOUT", 7: "SQUAD_ERR_WORKSPACE"}
+           4: "SQUAD_ERR_UNSUPPORTED", 5: "SQUAD_ERR_CUDA", 6: "SQUAD_ERR_TIMEOUT", 7: "SQUAD_ERR_WORKSPACE",
+           8: "SQUAD_ERR_INDEX"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None

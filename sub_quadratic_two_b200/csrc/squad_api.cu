@@ -18,6 +18,8 @@
 #include "squad_fwd_tc.cuh"
 #include "squad_simt.cuh"
 #include "tmap_cache.h"
+#include "sp_plan.h"
+#include "squad_sp.cuh"
 
 namespace {
 
@@ -49,7 +51,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
-  bool fwd_attr_set[2] = {};     // [D=64/128]
+  bool fwd_attr_set[2][2] = {};  // [D=64/128][packed]
   bool fused_attr_set[2][2] = {};   // [D=64/128][out_f32]
 };
 
@@ -194,11 +196,11 @@ sq::PassArgs pass_args(const Geom& g, void* out, float* lse) {
   return pa;
 }
 
-template <int D>
+template <int D, bool PACKED>
 squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap* m, const sq::FwdArgs& a, cudaStream_t st) {
   using Lay = sq::FwdLayout<D>;
-  auto kern = sq::squad_fwd_tc_kernel<D>;
-  bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0];
+  auto kern = sq::squad_fwd_tc_kernel<D, PACKED>;
+  bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0][PACKED ? 1 : 0];
   if (!attr) {
     SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
     attr = true;
@@ -259,8 +261,9 @@ squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, cons
   a.err = ds->err;
   a.timeout_ns = kWaitTimeoutNs;
   if (mode == sq::FWD_FUSED) SQ_CUDA(cudaMemsetAsync(counters, 0, size_t(a.bh) * sizeof(uint32_t), st));
-  if (d == 128) return launch_fwd_tc_t<128>(ds, m, a, st);
-  return launch_fwd_tc_t<64>(ds, m, a, st);
+  const bool packed = p.g1.pk > 1 || p.g2.pk > 1;
+  if (d == 128) return packed ? launch_fwd_tc_t<128, true>(ds, m, a, st) : launch_fwd_tc_t<128, false>(ds, m, a, st);
+  return packed ? launch_fwd_tc_t<64, true>(ds, m, a, st) : launch_fwd_tc_t<64, false>(ds, m, a, st);
 }
 
 dim3 simt_grid(const Geom& g) { return dim3(unsigned(g.bh * g.probs), unsigned(sq::ceil_div(g.L, sq::kSimtWarps))); }
@@ -665,7 +668,7 @@ squad_status squad_poll_device_error(void* stream) {
   if (v != 0) {
     const int zero = 0;
     SQ_CUDA(cudaMemcpyToSymbol(g_squad_dev_err, &zero, sizeof(int)));
-    return SQUAD_ERR_TIMEOUT;
+    return v == 2 ? SQUAD_ERR_INDEX : SQUAD_ERR_TIMEOUT;
   }
   return SQUAD_OK;
 }
@@ -680,6 +683,7 @@ const char* squad_strerror(int status) {
     case SQUAD_ERR_CUDA: return "CUDA error";
     case SQUAD_ERR_TIMEOUT: return "device wait timed out";
     case SQUAD_ERR_WORKSPACE: return "workspace missing or too small";
+    case SQUAD_ERR_INDEX: return "a row index given to a shuffle was out of range";
   }
   return "unknown status";
 }
@@ -888,6 +892,149 @@ squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int*
     up = dval;
     acc ^= 1;
   }
+  return SQUAD_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- sequence-parallel forward
+// Plan (host only) and row shuffles around the two all-to-alls; see sp_plan.h.
+
+namespace {
+
+squad_status sp_plan_of(const squad_desc* d, int G, int rank, sq::SpPlan& p) {
+  if (d == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (G < 1 || G > sq::kSpMaxPeers || rank < 0 || rank >= G) return SQUAD_ERR_INVALID_ARG;
+  Plan base;
+  squad_status s = make_plan(d, &base, false);
+  if (s != SQUAD_OK) return s;
+  if (d->T % d->tT || d->H % d->tH || d->W % d->tW) return SQUAD_ERR_SHAPE;
+  const sq::SpShape sh{d->T, d->H, d->W, d->tT, d->tH, d->tW, G, rank};
+  if (!sq::plan_sp(sh, p)) return SQUAD_ERR_UNSUPPORTED;
+  return SQUAD_OK;
+}
+
+squad_status sp_shuffle_args(int ntensors, int slices, int rows_in, int rows_out, int row_bytes, int G,
+                             const int* counts, sq::SpShuffleArgs* a) {
+  if (ntensors < 1 || ntensors > sq::kSpMaxTensors || slices < 1 || rows_in < 0 || rows_out < 0 || row_bytes <= 0 ||
+      row_bytes % 16 != 0 || G < 1 || G > sq::kSpMaxPeers || counts == nullptr)
+    return SQUAD_ERR_INVALID_ARG;
+  *a = sq::SpShuffleArgs{};
+  a->ntensors = ntensors;
+  a->slices = slices;
+  a->rows_in = rows_in;
+  a->rows_out = rows_out;
+  a->row_bytes = row_bytes;
+  a->G = G;
+  long long at = 0;
+  for (int q = 0; q < G; ++q) {
+    if (counts[q] < 0) return SQUAD_ERR_INVALID_ARG;
+    a->prefix[q] = int(at);
+    at += counts[q];
+  }
+  a->prefix[G] = int(at);
+  if ((long long)ntensors * slices * (at > rows_out ? at : rows_out) * row_bytes >= (1ll << 40) || at >= (1ll << 31))
+    return SQUAD_ERR_SHAPE;
+  return SQUAD_OK;
+}
+
+unsigned sp_blocks(long long chunks, int sms) {
+  const long long b = (chunks + 255) / 256;
+  const long long cap = 8ll * sms;
+  return unsigned(b < 1 ? 1 : b > cap ? cap : b);
+}
+
+}  // namespace
+
+extern "C" {
+
+squad_status squad_sp_plan_info(const squad_desc* desc, int G, int rank, int* info) {
+  if (info == nullptr) return SQUAD_ERR_INVALID_ARG;
+  sq::SpPlan p;
+  squad_status s = sp_plan_of(desc, G, rank, p);
+  if (s != SQUAD_OK) return s;
+  info[0] = p.t0;
+  info[1] = p.T;
+  info[2] = p.n_local;
+  info[3] = p.n_pos;
+  info[4] = p.p0[rank];
+  info[5] = p.np[rank];
+  info[6] = p.w;
+  info[7] = p.m;
+  return SQUAD_OK;
+}
+
+squad_status squad_sp_plan_maps(const squad_desc* desc, int G, int rank, int* counts, int* send1, int* recv1_src,
+                                int* recv1_row, int* send2, int* recv2_src, int* recv2_row) {
+  for (const void* ptr : {static_cast<const void*>(counts), static_cast<const void*>(send1),
+                          static_cast<const void*>(recv1_src), static_cast<const void*>(recv1_row),
+                          static_cast<const void*>(send2), static_cast<const void*>(recv2_src),
+                          static_cast<const void*>(recv2_row)})
+    if (ptr == nullptr) return SQUAD_ERR_INVALID_ARG;
+  sq::SpPlan p;
+  squad_status s = sp_plan_of(desc, G, rank, p);
+  if (s != SQUAD_OK) return s;
+  for (int q = 0; q < G; ++q) {
+    counts[q] = p.send1_count[q];
+    counts[G + q] = p.recv1_count[q];
+    counts[2 * G + q] = p.send2_count[q];
+    counts[3 * G + q] = p.recv2_count[q];
+  }
+  std::memcpy(send1, p.send1.data(), sizeof(int) * p.send1.size());
+  std::memcpy(recv1_src, p.recv1_src.data(), sizeof(int) * p.recv1_src.size());
+  std::memcpy(recv1_row, p.recv1_row.data(), sizeof(int) * p.recv1_row.size());
+  std::memcpy(send2, p.send2.data(), sizeof(int) * p.send2.size());
+  std::memcpy(recv2_src, p.recv2_src.data(), sizeof(int) * p.recv2_src.size());
+  std::memcpy(recv2_row, p.recv2_row.data(), sizeof(int) * p.recv2_row.size());
+  return SQUAD_OK;
+}
+
+squad_status squad_sp_pack(const void* const* srcs, int ntensors, int slices, int rows_in, int row_bytes, int G,
+                           const int* counts, const int* idx, void* dst, void* stream) {
+  sq::SpShuffleArgs a;
+  squad_status s = sp_shuffle_args(ntensors, slices, rows_in, 0, row_bytes, G, counts, &a);
+  if (s != SQUAD_OK) return s;
+  if (srcs == nullptr || idx == nullptr || dst == nullptr) return SQUAD_ERR_INVALID_ARG;
+  for (int t = 0; t < ntensors; ++t) {
+    if (srcs[t] == nullptr) return SQUAD_ERR_INVALID_ARG;
+    if (!aligned16(srcs[t])) return SQUAD_ERR_ALIGN;
+    a.src[t] = static_cast<const uint8_t*>(srcs[t]);
+  }
+  if (!aligned16(dst) || (reinterpret_cast<uintptr_t>(idx) & 3u)) return SQUAD_ERR_ALIGN;
+  a.dst[0] = static_cast<uint8_t*>(dst);
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  a.err = ds->err;
+  const long long chunks = (long long)ntensors * slices * a.prefix[G] * (row_bytes / 16);
+  if (chunks == 0) return SQUAD_OK;
+  sq::sp_pack_kernel<<<sp_blocks(chunks, ds->sms), 256, 0, static_cast<cudaStream_t>(stream)>>>(a, idx);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
+squad_status squad_sp_unpack(const void* src, int ntensors, int slices, int rows_out, int row_bytes, int G,
+                             const int* counts, const int* src_rank, const int* src_row, void* const* dsts,
+                             void* stream) {
+  sq::SpShuffleArgs a;
+  squad_status s = sp_shuffle_args(ntensors, slices, 0, rows_out, row_bytes, G, counts, &a);
+  if (s != SQUAD_OK) return s;
+  if (src == nullptr || src_rank == nullptr || src_row == nullptr || dsts == nullptr) return SQUAD_ERR_INVALID_ARG;
+  if (!aligned16(src) || (reinterpret_cast<uintptr_t>(src_rank) & 3u) || (reinterpret_cast<uintptr_t>(src_row) & 3u))
+    return SQUAD_ERR_ALIGN;
+  a.src[0] = static_cast<const uint8_t*>(src);
+  for (int t = 0; t < ntensors; ++t) {
+    if (dsts[t] == nullptr) return SQUAD_ERR_INVALID_ARG;
+    if (!aligned16(dsts[t])) return SQUAD_ERR_ALIGN;
+    a.dst[t] = static_cast<uint8_t*>(dsts[t]);
+  }
+  DeviceState* ds = nullptr;
+  if ((s = device_state(&ds)) != SQUAD_OK) return s;
+  a.err = ds->err;
+  const long long chunks = (long long)ntensors * slices * rows_out * (row_bytes / 16);
+  if (chunks == 0) return SQUAD_OK;
+  sq::sp_unpack_kernel<<<sp_blocks(chunks, ds->sms), 256, 0, static_cast<cudaStream_t>(stream)>>>(a, src_rank,
+                                                                                                  src_row);
+  SQ_CUDA(cudaGetLastError());
   return SQUAD_OK;
 }
 

@@ -186,7 +186,9 @@ __device__ __forceinline__ bool wait_counter(const uint32_t* c, uint32_t target,
   }
 }
 
-template <int D>
+// PACKED: the geometry may pack several problems to a box (a per-row key mask then
+// applies); the two-pass operator never packs, and its kernel is smaller without it.
+template <int D, bool PACKED>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     squad_fwd_tc_kernel(const __grid_constant__ CUtensorMap m0, const __grid_constant__ CUtensorMap m1,
                         const __grid_constant__ CUtensorMap m2, const __grid_constant__ CUtensorMap m3,
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const Geom& g = args.ps[it.pass].g;
         int tok = row < tile_valid_rows(g, J.qt) ? J.base + tile_row_offset(g, J.qt, row) : -1;
         // packed geometry: a row past the packed digit's extent is a zero-filled row
-        if (g.pk > 1 && J.j0 + pack_id(g, row) >= g.pk_ext) tok = -1;
+        if (PACKED && g.pk > 1 && J.j0 + pack_id(g, row) >= g.pk_ext) tok = -1;
         return SJob{i, it.pass, J.qt, J.base, tok};
       }
       return SJob{args.total_items, 0, 0, 0, -1};
@@ -480,7 +482,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (32 * j + e >= lim) r[32 * j + e] = 0xff800000u;
           }
         }
-        if (g.pk > 1) {
+        if (PACKED && g.pk > 1) {
           // packed problems: keys of other problems in the box -> -inf. This row's problem
           // holds runs of pk_rowdiv columns, one run every pk * pk_rowdiv columns.
           const int R = g.pk_rowdiv;

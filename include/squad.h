@@ -156,8 +156,10 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
  * its values are the output of pass j-1 (v for j = 1); q, k and the scale are
  * those of every pass; the result is the output of pass k. ntiles = 1 is
  * the operator of squad_attn_fwd with tile t_1. Cost: 4 n d (|t_1| +
- * |t_2|/|t_1| + ... + n/|t_{k-1}|) FLOPs per (batch, head). Each pass is one
- * launch of the kernels above (no fused hand-off between passes). On bf16 the
+ * |t_2|/|t_1| + ... + n/|t_{k-1}|) FLOPs per (batch, head). On bf16 with a
+ * workspace the k passes run in one launch, pass j of a (batch, head) starting
+ * once pass j-1 of it is done (the results are bitwise those of one launch per
+ * pass); otherwise each pass is one launch. On bf16 the
  * forward packs the problems of a pass several to a tensor-core box when they
  * have at most 64 tokens and the problem box has an extent-1 dimension (a
  * per-row key mask keeps them apart); the results then equal the unpacked
@@ -165,12 +167,28 @@ squad_status squad_attn_bwd(const squad_desc* desc, const void* q, const void* k
  * along W) must be at most 128 tokens (else SQUAD_ERR_UNSUPPORTED); tiles
  * that do not nest give SQUAD_ERR_SHAPE. */
 
+/* Bytes of workspace squad_attn_multi_fwd needs. save_inter != 0 (the caller
+ * passes inter): one uint32 counter per (pass 2..k, batch, head), for the
+ * one-launch bf16 forward. save_inter == 0 (inter NULL): first the k-1
+ * intermediate outputs, then the counters. Each part is 256-byte aligned. */
+squad_status squad_attn_multi_fwd_workspace_size(const squad_desc* desc, int ntiles, const int* tiles,
+                                                 int save_inter, size_t* bytes);
+
 /* Forward. inter: ntiles consecutive [B, heads, n, d] tensors of the input
- * dtype receiving the outputs of passes 1..k-1 (required: each is the next
- * pass's values, and the backward reads them). lse: k consecutive [B, heads, n]
- * fp32 (natural log), or NULL. o, inter, lse are written, nothing else. */
+ * dtype receiving the outputs of passes 1..k-1 (each is the next pass's values,
+ * and the backward reads them), or NULL for inference: they then live in the
+ * workspace, and on bf16 each row leaves L2 without being written back once
+ * the next pass has read it (when its problem fits one box). lse: k
+ * consecutive [B, heads, n] fp32 (natural log), or NULL. workspace: device,
+ * 16-byte aligned, at least squad_attn_multi_fwd_workspace_size bytes for the
+ * same save_inter (else SQUAD_ERR_WORKSPACE), owned by the caller and
+ * overwritten, not read; NULL (allowed only with inter) runs one launch per
+ * pass; it must not be shared with a call in flight on another stream. On f32
+ * only its intermediate part is used. o, inter, lse (and the workspace) are
+ * written, nothing else. */
 squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
-                                  const void* k, const void* v, void* o, void* inter, float* lse, void* stream);
+                                  const void* k, const void* v, void* o, void* inter, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace squad_attn_multi_bwd needs: two upstream-gradient
  * tensors of the input dtype, four fp32 [B, heads, n, d] accumulators and one

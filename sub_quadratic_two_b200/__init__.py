@@ -23,6 +23,7 @@ __all__ = [
     "SquadError", "attention", "squad_attn_fwd", "squad_attn_bwd", "workspace_size",
     "poll_device_error", "library_path", "load_library", "SQUAD_F32", "SQUAD_BF16", "squad_attn_fwd_pass",
     "plan_info", "make_desc", "attention_multi", "squad_attn_multi_fwd", "squad_attn_multi_bwd",
+    "multi_fwd_workspace_size",
     "tmap_cache_stats",
 ]
 
@@ -72,7 +73,9 @@ def load_library():
         lib.squad_attn_fwd_pass.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, fp, vp]
         lib.squad_plan_info.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         ip = ctypes.POINTER(ctypes.c_int)
-        lib.squad_attn_multi_fwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp]
+        lib.squad_attn_multi_fwd_workspace_size.argtypes = [dp, ctypes.c_int, ip, ctypes.c_int,
+                                                            ctypes.POINTER(ctypes.c_size_t)]
+        lib.squad_attn_multi_fwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp, sz, vp]
         lib.squad_attn_multi_bwd_workspace_size.argtypes = [dp, ctypes.c_int, ip, ctypes.POINTER(ctypes.c_size_t)]
         lib.squad_attn_multi_bwd.argtypes = [dp, ctypes.c_int, ip, vp, vp, vp, vp, vp, fp, vp, vp, vp, vp, vp,
                                              sz, vp]
@@ -82,7 +85,7 @@ def load_library():
         lib.squad_strerror.argtypes = [ctypes.c_int]
         lib.squad_strerror.restype = ctypes.c_char_p
         for f in ("squad_attn_workspace_size", "squad_attn_fwd", "squad_attn_bwd", "squad_poll_device_error",
-                  "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_multi_fwd",
+                  "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_multi_fwd_workspace_size", "squad_attn_multi_fwd",
                   "squad_attn_multi_bwd_workspace_size", "squad_attn_multi_bwd",
                   "squad_last_cuda_error", "squad_version", "squad_tmap_cache_stats"):
             getattr(lib, f).restype = ctypes.c_int
@@ -321,23 +324,45 @@ def _tiles_arg(tiles: Sequence[Sequence[int]]):
 
 
 def squad_attn_multi_fwd(q, k, v, grid, tiles, scale: Optional[float] = None,
-                         stream: Optional[torch.cuda.Stream] = None):
+                         stream: Optional[torch.cuda.Stream] = None, one_launch: bool = True,
+                         save: bool = True, out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None):
     """k = len(tiles) + 1 passes over nested tiles (innermost first) through the C ABI.
 
     Returns (o, inter, lse): inter is [k-1, B, heads, n, d] (outputs of passes
-    1..k-1), lse is [k, B, heads, n] fp32.
+    1..k-1), lse is [k, B, heads, n] fp32. one_launch: on bf16, run all passes in
+    one launch (passes a counter workspace); False runs one launch per pass.
+    save=False (inference): the intermediate outputs and the LSE are not kept
+    (inter and lse are None; the intermediates live in the workspace and, on bf16,
+    leave L2 without a write-back once read). out / workspace: optional
+    preallocated output and workspace (at least the size the library asks for).
     """
     lib = load_library()
     _check_inputs(q, k, v)
     desc = make_desc(q, grid, tiles[0], scale)
     nt, tarr = _tiles_arg(tiles)
-    o = torch.empty_like(q)
-    inter = torch.empty((nt,) + tuple(q.shape), device=q.device, dtype=q.dtype)
-    lse = torch.empty((nt + 1,) + tuple(q.shape[:3]), device=q.device, dtype=torch.float32)
+    if out is not None:
+        _check_aux(out, tuple(q.shape), q.dtype, q.device, "out")
+    o = torch.empty_like(q) if out is None else out
+    inter = torch.empty((nt,) + tuple(q.shape), device=q.device, dtype=q.dtype) if save else None
+    lse = torch.empty((nt + 1,) + tuple(q.shape[:3]), device=q.device, dtype=torch.float32) if save else None
+    ws, ws_n = None, 0
+    if one_launch or not save:
+        nb = ctypes.c_size_t(0)
+        _check(lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(desc), nt, tarr, int(save), ctypes.byref(nb)),
+               "squad_attn_multi_fwd_workspace_size")
+        ws_n = int(nb.value)
+        if workspace is not None:
+            if workspace.device != q.device or not workspace.is_contiguous() or workspace.numel() * workspace.element_size() < ws_n:
+                raise ValueError(f"workspace must be a contiguous tensor of at least {ws_n} bytes on {q.device}")
+            ws = workspace
+            ws_n = workspace.numel() * workspace.element_size()
+        else:
+            ws = torch.empty(ws_n, device=q.device, dtype=torch.uint8)
     with torch.cuda.device(q.device):
         st = _stream_handle(stream, q.device)
         _check(lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, tarr, _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                        _ptr(inter), _ptr(lse), st), "squad_attn_multi_fwd")
+                                        _ptr(inter), _ptr(lse), _ptr(ws), ws_n, st), "squad_attn_multi_fwd")
     return o, inter, lse
 
 
@@ -362,6 +387,17 @@ def squad_attn_multi_bwd(q, k, v, o, inter, lse, dout, grid, tiles, scale: Optio
                                         _ptr(dk), _ptr(dv), _ptr(ws), int(ws_bytes.value), st),
                "squad_attn_multi_bwd")
     return dq, dk, dv
+
+
+def multi_fwd_workspace_size(q: torch.Tensor, grid, tiles, save: bool = True, scale: Optional[float] = None) -> int:
+    """Bytes of workspace squad_attn_multi_fwd asks for (save: the caller keeps the intermediates)."""
+    lib = load_library()
+    desc = make_desc(q, grid, tiles[0], scale)
+    nt, tarr = _tiles_arg(tiles)
+    nb = ctypes.c_size_t(0)
+    _check(lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(desc), nt, tarr, int(save), ctypes.byref(nb)),
+           "squad_attn_multi_fwd_workspace_size")
+    return int(nb.value)
 
 
 class _SquadAttentionMulti(torch.autograd.Function):

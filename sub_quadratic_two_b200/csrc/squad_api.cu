@@ -29,6 +29,7 @@ constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s per wait: far above any legitimate wait
 constexpr int kFusedLag = 2;  // heads between a local pass and its global pass (see decode_item)
+constexpr int kMultiLag = 2;  // heads between pass j-1 and pass j of a head in the k-pass launch
 
 thread_local int t_last_cuda = 0;
 
@@ -197,7 +198,7 @@ sq::PassArgs pass_args(const Geom& g, void* out, float* lse) {
 }
 
 template <int D, bool PACKED>
-squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap* m, const sq::FwdArgs& a, cudaStream_t st) {
+squad_status launch_fwd_tc_t(DeviceState* ds, const sq::FwdMaps& m, const sq::FwdArgs& a, cudaStream_t st) {
   using Lay = sq::FwdLayout<D>;
   auto kern = sq::squad_fwd_tc_kernel<D, PACKED>;
   bool& attr = ds->fwd_attr_set[D == 128 ? 1 : 0][PACKED ? 1 : 0];
@@ -212,12 +213,12 @@ squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap* m, const sq::Fw
   cfg.dynamicSmemBytes = Lay::ALLOC;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
-  // The fused launch has CTAs wait on other CTAs' progress: require co-residency.
+  // Chained passes have CTAs wait on other CTAs' progress: require co-residency.
   attrs[0].id = cudaLaunchAttributeCooperative;
-  attrs[0].val.cooperative = a.mode == sq::FWD_FUSED ? 1 : 0;
+  attrs[0].val.cooperative = (a.mode == sq::FWD_FUSED || a.mode == sq::FWD_MULTI) ? 1 : 0;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  SQ_CUDA(cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], a));
+  SQ_CUDA(cudaLaunchKernelEx(&cfg, kern, m, a));
   return SQUAD_OK;
 }
 
@@ -226,7 +227,8 @@ squad_status launch_fwd_tc_t(DeviceState* ds, const CUtensorMap* m, const sq::Fw
 squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, const void* q, const void* k,
                            const void* val1, void* out1, float* lse1, const void* val2, void* out2, float* lse2,
                            uint32_t* counters, const void* discard, cudaStream_t st) {
-  CUtensorMap m[8];
+  sq::FwdMaps maps;
+  CUtensorMap* m = maps.m;
   squad_status s;
   const bool do1 = mode != sq::FWD_GLOBAL, do2 = mode != sq::FWD_LOCAL;
   if (do1) {
@@ -245,7 +247,9 @@ squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, cons
     if (!do1) m[i] = m[4 + i];
     if (!do2) m[4 + i] = m[i];
   }
+  for (int i = 8; i < 4 * sq::kMaxFwdPasses; ++i) m[i] = m[i & 7];  // unused
   sq::FwdArgs a{};
+  a.npass = 2;
   a.ps[0] = pass_args(p.g1, out1, lse1);
   a.ps[1] = pass_args(p.g2, out2, lse2);
   a.mode = mode;
@@ -257,13 +261,13 @@ squad_status launch_fwd_tc(DeviceState* ds, int d, int mode, const Plan& p, cons
   a.f_n12 = sq::make_fastdiv(uint32_t(a.ps[0].pairs_per_bh + a.ps[1].pairs_per_bh));
   a.scale_log2 = p.scale * 1.4426950408889634f;
   a.counters = counters;
-  a.discard_base = static_cast<const uint8_t*>(discard);
+  a.ps[1].discard = static_cast<const uint8_t*>(discard);
   a.err = ds->err;
   a.timeout_ns = kWaitTimeoutNs;
   if (mode == sq::FWD_FUSED) SQ_CUDA(cudaMemsetAsync(counters, 0, size_t(a.bh) * sizeof(uint32_t), st));
   const bool packed = p.g1.pk > 1 || p.g2.pk > 1;
-  if (d == 128) return packed ? launch_fwd_tc_t<128, true>(ds, m, a, st) : launch_fwd_tc_t<128, false>(ds, m, a, st);
-  return packed ? launch_fwd_tc_t<64, true>(ds, m, a, st) : launch_fwd_tc_t<64, false>(ds, m, a, st);
+  if (d == 128) return packed ? launch_fwd_tc_t<128, true>(ds, maps, a, st) : launch_fwd_tc_t<128, false>(ds, maps, a, st);
+  return packed ? launch_fwd_tc_t<64, true>(ds, maps, a, st) : launch_fwd_tc_t<64, false>(ds, maps, a, st);
 }
 
 dim3 simt_grid(const Geom& g) { return dim3(unsigned(g.bh * g.probs), unsigned(sq::ceil_div(g.L, sq::kSimtWarps))); }
@@ -706,7 +710,8 @@ int squad_version(void) { return kVersion; }
 // t_{j-1}-window; its values are the previous pass's output. The pages name composing
 // more than two passes as an outlook (gist.science technical summary, Significance and
 // Claims); k = 2 is the operator above. Each pass runs on the same kernels as the two
-// SQuad passes, one launch per pass.
+// SQuad passes: on bf16 with a workspace, all k passes in one launch (pass j of a head
+// starts once pass j-1 of that head is done everywhere), else one launch per pass.
 
 namespace {
 
@@ -747,6 +752,68 @@ squad_status make_multi_plan(const squad_desc* d, int ntiles, const int* tiles, 
     mp->gf[j - 1] = gf;
   }
   return SQUAD_OK;
+}
+
+// Forward workspace: [outputs of passes 1..k-1, only when the caller passes no inter]
+// [finished jobs per (pass, batch, head) for passes 2..k].
+size_t multi_fwd_inter_bytes(const MultiPlan& mp, const squad_desc* d) {
+  return align256(size_t(mp.k - 1) * mp.base.rows * d->d * mp.base.elem);
+}
+size_t multi_fwd_counter_bytes(const MultiPlan& mp) {
+  return align256(size_t(mp.k - 1) * mp.g[0].bh * sizeof(uint32_t));
+}
+
+// All k passes of the bf16 forward in one cooperative launch (FWD_MULTI item order, see
+// decode_item): val[j] / out[j] / lse[j] are pass j's values, output and LSE.
+squad_status launch_fwd_multi(DeviceState* ds, int d, const MultiPlan& mp, const void* q, const void* k,
+                              const void* const* val, void* const* out, float* const* lse, uint32_t* counters,
+                              bool drop_inter, cudaStream_t st) {
+  sq::FwdMaps maps;
+  sq::FwdArgs a{};
+  squad_status s;
+  const int np = mp.k;
+  if (np > sq::kMaxFwdPasses) return SQUAD_ERR_UNSUPPORTED;
+  bool packed = false;
+  for (int j = 0; j < np; ++j) {
+    const Geom& g = mp.gf[j];
+    CUtensorMap* m = &maps.m[4 * j];
+    if ((s = encode_map(&m[0], q, g, d, mp.base.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[1], k, g, d, mp.base.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[2], val[j], g, d, mp.base.rows)) != SQUAD_OK) return s;
+    if ((s = encode_map(&m[3], out[j], g, d, mp.base.rows)) != SQUAD_OK) return s;
+    a.ps[j] = pass_args(g, out[j], lse[j]);
+    // scratch values (a previous pass's output nobody else reads) leave L2 once read
+    if (drop_inter && j > 0 && (reinterpret_cast<uintptr_t>(val[j]) & 127u) == 0)
+      a.ps[j].discard = static_cast<const uint8_t*>(val[j]);
+    packed = packed || g.pk > 1;
+  }
+  for (int i = 4 * np; i < 4 * sq::kMaxFwdPasses; ++i) maps.m[i] = maps.m[i % (4 * np)];  // unused
+  a.mode = sq::FWD_MULTI;
+  a.npass = np;
+  a.bh = mp.gf[0].bh;
+  a.lag = kMultiLag < a.bh ? kMultiLag : a.bh;
+  a.pref[0] = 0;
+  for (int j = 0; j < np; ++j) a.pref[j + 1] = a.pref[j] + a.ps[j].pairs_per_bh;
+  a.total_items = a.bh * a.pref[np];
+  // blocks 0 .. bh-1 + (np-1)*lag; block b holds pass j of head b - j*lag while that head
+  // exists, so blocks (np-1)*lag .. bh-1 hold every pass
+  const int first_full = (np - 1) * a.lag;
+  a.nmid = a.bh > first_full ? a.bh - first_full : 0;
+  a.lead_items = 0;
+  for (int b = 0; b < first_full; ++b)
+    for (int j = 0; j < np; ++j) {
+      const int h = b - j * a.lag;
+      if (h >= 0 && h < a.bh) a.lead_items += a.ps[j].pairs_per_bh;
+    }
+  a.f_full = sq::make_fastdiv(uint32_t(a.pref[np]));
+  a.f_n1 = a.f_n2 = a.f_n12 = a.f_full;  // unused in this mode
+  a.scale_log2 = mp.base.scale * 1.4426950408889634f;
+  a.counters = counters;
+  a.err = ds->err;
+  a.timeout_ns = kWaitTimeoutNs;
+  SQ_CUDA(cudaMemsetAsync(counters, 0, size_t(np - 1) * a.bh * sizeof(uint32_t), st));
+  if (d == 128) return packed ? launch_fwd_tc_t<128, true>(ds, maps, a, st) : launch_fwd_tc_t<128, false>(ds, maps, a, st);
+  return packed ? launch_fwd_tc_t<64, true>(ds, maps, a, st) : launch_fwd_tc_t<64, false>(ds, maps, a, st);
 }
 
 // Backward workspace: two upstream gradients (dtype) used in turn, two fp32 dQ and two
@@ -805,20 +872,48 @@ squad_status squad_attn_multi_bwd_workspace_size(const squad_desc* desc, int nti
   return SQUAD_OK;
 }
 
-squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
-                                  const void* k, const void* v, void* o, void* inter, float* lse, void* stream) {
+squad_status squad_attn_multi_fwd_workspace_size(const squad_desc* desc, int ntiles, const int* tiles,
+                                                 int save_inter, size_t* bytes) {
+  if (bytes == nullptr) return SQUAD_ERR_INVALID_ARG;
   MultiPlan mp;
   squad_status s = make_multi_plan(desc, ntiles, tiles, &mp);
   if (s != SQUAD_OK) return s;
-  for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(inter)})
+  *bytes = (save_inter ? 0 : multi_fwd_inter_bytes(mp, desc)) + multi_fwd_counter_bytes(mp);
+  return SQUAD_OK;
+}
+
+squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int* tiles, const void* q,
+                                  const void* k, const void* v, void* o, void* inter, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  MultiPlan mp;
+  squad_status s = make_multi_plan(desc, ntiles, tiles, &mp);
+  if (s != SQUAD_OK) return s;
+  for (const void* ptr : {q, k, v, static_cast<const void*>(o)})
     if (ptr == nullptr) return SQUAD_ERR_INVALID_ARG;
   for (const void* ptr : {q, k, v, static_cast<const void*>(o), static_cast<const void*>(inter),
-                          static_cast<const void*>(lse)})
+                          static_cast<const void*>(lse), static_cast<const void*>(workspace)})
     if (!aligned16(ptr)) return SQUAD_ERR_ALIGN;
+  const bool save = inter != nullptr;
+  if (!save && workspace == nullptr) return SQUAD_ERR_WORKSPACE;
+  const size_t inter_ws = save ? 0 : multi_fwd_inter_bytes(mp, desc);
+  if (workspace != nullptr && workspace_bytes < inter_ws + multi_fwd_counter_bytes(mp)) return SQUAD_ERR_WORKSPACE;
+  if (!save) inter = workspace;
   DeviceState* ds = nullptr;
   if ((s = device_state(&ds)) != SQUAD_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t big = size_t(mp.base.rows) * desc->d * mp.base.elem;
+  if (desc->dtype == SQUAD_BF16 && workspace != nullptr) {
+    const void* vals[sq::kMaxFwdPasses];
+    void* outs[sq::kMaxFwdPasses];
+    float* lses[sq::kMaxFwdPasses];
+    for (int j = 0; j < mp.k; ++j) {
+      outs[j] = j == mp.k - 1 ? o : static_cast<uint8_t*>(inter) + big * j;
+      vals[j] = j == 0 ? v : outs[j - 1];
+      lses[j] = lse == nullptr ? nullptr : lse + size_t(mp.base.rows) * j;
+    }
+    uint32_t* counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + inter_ws);
+    return launch_fwd_multi(ds, desc->d, mp, q, k, vals, outs, lses, counters, !save, st);
+  }
   const void* val = v;
   for (int j = 1; j <= mp.k; ++j) {
     void* out = j == mp.k ? o : static_cast<uint8_t*>(inter) + big * (j - 1);

@@ -25,7 +25,8 @@
 //   warps 9,11 one thread each issues tcgen05.mma for one softmax warpgroup:
 //              S = Q K^T (both operands K-major) and O += P V (P read from TMEM,
 //              V MN-major)
-//   warp 10    fused launch: publishes per-head completion of the local pass
+//   warp 10    chained passes: publishes per-(pass, head) completion of the passes
+//              other than the last
 // The softmax warpgroups write their output rows (through a per-warp transpose patch,
 // so that stores are whole 128-byte lines) and, for inference, drop the consumed
 // local-pass rows from L2.
@@ -41,26 +42,34 @@
 
 namespace sq {
 
-enum { FWD_LOCAL = 1, FWD_GLOBAL = 2, FWD_FUSED = 3 };
+enum { FWD_LOCAL = 1, FWD_GLOBAL = 2, FWD_FUSED = 3, FWD_MULTI = 4 };
+constexpr int kMaxFwdPasses = 5;
 
 struct PassArgs {
   Geom g;
   void* out;          // [rows, D] bf16 output of this pass
   float* lse;         // natural-log LSE of this pass, or nullptr
+  const uint8_t* discard;  // this pass's values when they are scratch read only here (dropped from L2
+                           // once read; rows 128-byte aligned), or nullptr
   int jobs_per_bh;    // problems per (batch, head) x boxes per problem
   int pairs_per_bh;   // ceil(jobs_per_bh / 2)
 };
 
 struct FwdArgs {
-  PassArgs ps[2];                // [0] local pass, [1] global pass
-  int mode;                      // FWD_LOCAL, FWD_GLOBAL or FWD_FUSED
+  PassArgs ps[kMaxFwdPasses];    // two-pass modes: [0] local pass, [1] global pass; FWD_MULTI: pass j at [j]
+  int mode;                      // FWD_LOCAL, FWD_GLOBAL, FWD_FUSED or FWD_MULTI
+  int npass;                     // passes (2 except in FWD_MULTI)
   int bh;                        // batch * heads
-  int lag;                       // FWD_FUSED: heads between a head's local pass and its global pass
+  int lag;                       // FWD_FUSED / FWD_MULTI: heads between pass j-1 of a head and its pass j
   int total_items;               // pairs over all (batch, head) and passes run
   FastDiv f_n1, f_n2, f_n12;     // ps[0].pairs_per_bh, ps[1].pairs_per_bh and their sum
+  // FWD_MULTI item order (see decode_item): pref[j] = pairs per head of passes before j,
+  // the items of the leading blocks, the number of full blocks and the full block size
+  int pref[kMaxFwdPasses + 1];
+  int lead_items, nmid;
+  FastDiv f_full;
   float scale_log2;              // softmax scale * log2(e)
-  uint32_t* counters;            // FWD_FUSED: finished local-pass jobs per (batch, head)
-  const uint8_t* discard_base;   // FWD_FUSED inference: local-pass output to drop from L2, or nullptr
+  uint32_t* counters;            // FWD_FUSED / FWD_MULTI: finished jobs per (pass, batch, head), passes < last
   int* err;
   uint64_t timeout_ns;
 };
@@ -93,6 +102,22 @@ struct Item {
   int pass, bh, pair;
 };
 
+// Tensor maps of up to kMaxFwdPasses passes, four per pass: Q, K, values, output.
+struct alignas(64) FwdMaps {
+  CUtensorMap m[4 * kMaxFwdPasses];
+};
+
+// FWD_MULTI: pairs of block b, which holds pass j of head b - j*lag for every pass whose
+// head exists.
+__device__ __forceinline__ int multi_block_items(const FwdArgs& a, int b) {
+  int s = 0;
+  for (int j = 0; j < a.npass; ++j) {
+    const int h = b - j * a.lag;
+    if (h >= 0 && h < a.bh) s += a.ps[j].pairs_per_bh;
+  }
+  return s;
+}
+
 
 // Work items in launch order. Fused: the local pass of heads 0..lag-1, then for each
 // later head h its local pass followed by the global pass of head h-lag, then the
@@ -100,6 +125,34 @@ struct Item {
 // to finish everywhere before its global pass needs it, while its Q, K and O1 are
 // still in L2.
 __device__ __forceinline__ Item decode_item(const FwdArgs& a, int i) {
+  if (a.mode == FWD_MULTI) {
+    // blocks in order; block b: pass 0 of head b, pass 1 of head b - lag, ... (each while
+    // that head exists), all pairs of one (pass, head) together. Full blocks, where every
+    // pass is present, are decoded directly; the leading and trailing ones by a scan.
+    const int N = a.pref[a.npass], first_full = (a.npass - 1) * a.lag;
+    int b, r;
+    if (i >= a.lead_items && i < a.lead_items + a.nmid * N) {
+      const int t = i - a.lead_items, q = fdiv(t, a.f_full);
+      b = first_full + q;
+      r = t - q * N;
+    } else {
+      int acc = i < a.lead_items ? 0 : a.lead_items + a.nmid * N;
+      b = i < a.lead_items ? 0 : first_full + a.nmid;
+      for (;; ++b) {
+        const int sz = multi_block_items(a, b);
+        if (i < acc + sz) break;
+        acc += sz;
+      }
+      r = i - acc;
+    }
+    for (int j = 0; j < a.npass; ++j) {
+      const int h = b - j * a.lag, n = a.ps[j].pairs_per_bh;
+      if (h < 0 || h >= a.bh) continue;
+      if (r < n) return {j, h, r};
+      r -= n;
+    }
+    return {a.npass - 1, 0, 0};  // not reached for i < total_items
+  }
   const int n1 = a.ps[0].pairs_per_bh, n2 = a.ps[1].pairs_per_bh;
   if (a.mode == FWD_LOCAL) {
     const int q = fdiv(i, a.f_n1);
@@ -118,6 +171,10 @@ __device__ __forceinline__ Item decode_item(const FwdArgs& a, int i) {
   if (blk < a.bh - lag) return r < n1 ? Item{0, blk + lag, r} : Item{1, blk, r - n1};
   const int t = j - (a.bh - lag) * (n1 + n2), q = fdiv(t, a.f_n2);
   return {1, a.bh - lag + q, t - q * n2};
+}
+
+__device__ __forceinline__ bool job_valid(const FwdArgs& a, const Item& it, int which) {
+  return 2 * it.pair + which < a.ps[it.pass].jobs_per_bh;
 }
 
 struct Job {
@@ -190,11 +247,7 @@ __device__ __forceinline__ bool wait_counter(const uint32_t* c, uint32_t target,
 // applies); the two-pass operator never packs, and its kernel is smaller without it.
 template <int D, bool PACKED>
 __global__ void __launch_bounds__(kFwdThreads, 1)
-    squad_fwd_tc_kernel(const __grid_constant__ CUtensorMap m0, const __grid_constant__ CUtensorMap m1,
-                        const __grid_constant__ CUtensorMap m2, const __grid_constant__ CUtensorMap m3,
-                        const __grid_constant__ CUtensorMap m4, const __grid_constant__ CUtensorMap m5,
-                        const __grid_constant__ CUtensorMap m6, const __grid_constant__ CUtensorMap m7,
-                        const __grid_constant__ FwdArgs args) {
+    squad_fwd_tc_kernel(const __grid_constant__ FwdMaps maps, const __grid_constant__ FwdArgs args) {
   using Lay = FwdLayout<D>;
   constexpr int DH = D / 64;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -204,11 +257,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::BAR_OFF + Lay::NBAR * 8 + 4);
   // per warpgroup: threads that finished writing their rows of local-pass jobs (monotonic)
   uint32_t* rows_done = reinterpret_cast<uint32_t*>(smem + Lay::BAR_OFF + Lay::NBAR * 8 + 8);
-  // tensor map of (pass, role), role: 0 Q, 1 K, 2 values (selected without a local array)
-  auto map_of = [&](int pass, int role) -> const CUtensorMap* {
-    const int i = pass * 4 + role;
-    return i == 0 ? &m0 : i == 1 ? &m1 : i == 2 ? &m2 : i == 3 ? &m3 : i == 4 ? &m4 : i == 5 ? &m5 : i == 6 ? &m6 : &m7;
-  };
+  // tensor map of (pass, role), role: 0 Q, 1 K, 2 values
+  auto map_of = [&](int pass, int role) -> const CUtensorMap* { return &maps.m[pass * 4 + role]; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t to = args.timeout_ns;
@@ -243,7 +293,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tmem_relinquish();
   }
   if (warp == 8 && lane == 0)
-    for (int i = 0; i < 8; ++i) prefetch_tmap(map_of(i >> 2, i & 3));
+    for (int i = 0; i < 4 * args.npass; ++i) prefetch_tmap(map_of(i >> 2, i & 3));
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -251,14 +301,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = *tmem_holder;
   const uint32_t sbase = smem_u32(smem);
   const bool fused = args.mode == FWD_FUSED;
+  // passes chained in one launch: pass j of a head reads the output of its pass j - 1
+  const bool chained = fused || args.mode == FWD_MULTI;
+  const int last_pass = args.npass - 1;
   // 384 threads at up to 168 registers each (the launch bound); no register reallocation
 
   if (warp == 8) {
     // ================================================================ TMA producer
     if (lane == 0) {
       uint32_t qc = 0, uc = 0;  // Q boxes and key/value ring entries issued
-      // L2 policies in the fused launch: the local pass's Q and K are read again by the
-      // global pass (keep), its V is not (drop first); the global pass is their last use.
+      // L2 policies when passes are chained: Q and K are read again by the next pass (keep)
+      // until the last pass; values are read once (drop first).
       const uint64_t pol_keep = make_policy_evict_last(), pol_drop = make_policy_evict_first();
       const uint64_t pol_norm = make_policy_evict_normal();
       bool ok = true;
@@ -271,9 +324,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const Job J[2] = {job_of(args, it, 0), job_of(args, it, 1)};
         const bool shared = J[1].valid && J[1].prob == J[0].prob;
         const uint32_t tx = uint32_t(g.box_rows) * D * 2;
-        bool dep_done = !(fused && it.pass == 1);
-        const uint64_t pol_qk = !fused ? pol_norm : it.pass == 0 ? pol_keep : pol_drop;
-        const uint64_t pol_v = !fused ? pol_norm : pol_drop;
+        bool dep_done = !(chained && it.pass > 0);
+        const uint64_t pol_qk = !chained ? pol_norm : it.pass < last_pass ? pol_keep : pol_drop;
+        const uint64_t pol_v = !chained ? pol_norm : pol_drop;
         for (int k = 0; ok && k < g.nt; ++k) {
           for (int x = 0; ok && x < 2; ++x) {
             if (!J[x].valid) continue;
@@ -304,9 +357,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               ++uc;
             }
             if (!dep_done) {
-              // the global pass of a head reads O1 only once the local pass of that head is complete
-              const uint32_t target = uint32_t(args.ps[0].jobs_per_bh);
-              if (!(ok = wait_counter(args.counters + it.bh, target, abort_flag, to))) break;
+              // pass j of a head reads the output of its pass j - 1 only once that is complete
+              const uint32_t target = uint32_t(args.ps[it.pass - 1].jobs_per_bh);
+              if (!(ok = wait_counter(args.counters + (it.pass - 1) * args.bh + it.bh, target, abort_flag, to)))
+                break;
               fence_async_global();
               dep_done = true;
             }
@@ -407,23 +461,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_wait_drain(&bars[F_DRAIN + x], 0, to);
     }
   } else if (warp == 10) {
-    // ================================================================ publisher (fused launch)
-    // Once all rows of a local-pass job are written (the warpgroup's 128 threads each add
-    // one to rows_done after their stores), make them visible at GPU scope and count the job for its
-    // head; the global pass of that head starts when its count is complete. Done here so
-    // the softmax warpgroups never wait for the fence.
-    if (fused && lane == 0) {
+    // ================================================================ publisher (chained passes)
+    // Once all rows of a job of a pass that is not the last are written (the warpgroup's
+    // 128 threads each add one to rows_done after their stores), make them visible at GPU
+    // scope and count the job for its (pass, head); the next pass of that head starts when
+    // its count is complete. Done here so the softmax warpgroups never wait for the fence.
+    if (chained && lane == 0) {
       uint32_t pub[2] = {0, 0};
       bool ok = true;
       for (int i = blockIdx.x; ok && i < args.total_items; i += gridDim.x) {
         const Item it = decode_item(args, i);
-        if (it.pass != 0) continue;
+        if (it.pass == last_pass) continue;
         for (int x = 0; ok && x < 2; ++x) {
-          if (!job_of(args, it, x).valid) continue;
+          if (!job_valid(args, it, x)) continue;
           ++pub[x];
           if (!(ok = wait_count_shared(&rows_done[x], 128u * pub[x], abort_flag, to))) break;
           fence_acq_rel_gpu();
-          red_release_gpu_add(args.counters + it.bh, 1u);
+          red_release_gpu_add(args.counters + it.pass * args.bh + it.bh, 1u);
         }
       }
     }
@@ -586,9 +640,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         int rtok[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) rtok[i] = __shfl_sync(0xffffffffu, cur.tok, 4 * i + lr);
-        // fused launch: O1 rows are read again by the global pass (keep); O rows are final (drop first)
-        const uint64_t pol_out = !fused ? make_policy_evict_normal()
-                                 : cur.pass == 0 ? make_policy_evict_last() : make_policy_evict_first();
+        // chained passes: an output read by the next pass is kept in L2, the last pass's dropped first
+        const uint64_t pol_out = !chained ? make_policy_evict_normal()
+                                 : cur.pass < last_pass ? make_policy_evict_last() : make_policy_evict_first();
         uint8_t* outb = static_cast<uint8_t*>(P.out);
 #pragma unroll 1
         for (int h = 0; h < D / 64; ++h) {
@@ -612,10 +666,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       tc_fence_before();
-      if (fused && cur.pass == 0) red_release_cta_shared_add(&rows_done[a], 1u);  // warp 10 publishes
-      if (live && args.discard_base != nullptr && cur.pass == 1 && g.nt == 1) {
-        // this row of the local-pass output was read once, as a value of this group: drop it from L2
-        const uint8_t* l1row = args.discard_base + tok * D * 2;
+      if (chained && cur.pass < last_pass) red_release_cta_shared_add(&rows_done[a], 1u);  // warp 10 publishes
+      if (live && P.discard != nullptr && g.nt == 1) {
+        // this row of the previous pass's output was read once, as a value of this group: drop it
+        const uint8_t* l1row = P.discard + tok * D * 2;
 #pragma unroll
         for (int l = 0; l < D * 2 / 128; ++l) discard_l2_line(l1row + l * 128);
       }

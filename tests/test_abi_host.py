@@ -144,9 +144,9 @@ def _tiles(*ts):
     return len(ts), (ctypes.c_int * len(flat))(*flat)
 
 
-def _mfwd(lib, desc, tiles, o=FAKE, inter=FAKE, lse=None):
+def _mfwd(lib, desc, tiles, o=FAKE, inter=FAKE, lse=None, ws=None, ws_bytes=0):
     nt, arr = tiles
-    return lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, arr, FAKE, FAKE, FAKE, o, inter, lse, None)
+    return lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, arr, FAKE, FAKE, FAKE, o, inter, lse, ws, ws_bytes, None)
 
 
 def test_multi_pass_argument_errors(lib):
@@ -155,9 +155,21 @@ def test_multi_pass_argument_errors(lib):
     assert _mfwd(lib, d, _tiles((1, 4, 4), (1, 2, 2))) == SHAPE          # outer tile smaller than inner
     assert _mfwd(lib, d, _tiles((1, 2, 2), (3, 4, 4))) == SHAPE          # 3 does not divide T=4
     assert _mfwd(lib, d, _tiles(*[(1, 1, 1)] * 5)) == UNSUPPORTED        # at most four tiles
-    assert lib.squad_attn_multi_fwd(ctypes.byref(d), 1, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None) == INVALID
-    assert _mfwd(lib, d, _tiles((1, 2, 2), (1, 4, 4)), inter=None) == INVALID
+    assert lib.squad_attn_multi_fwd(ctypes.byref(d), 1, None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0,
+                                    None) == INVALID
     assert _mfwd(lib, d, _tiles((1, 2, 2), (1, 4, 4)), o=MISALIGNED) == ALIGN
+    # the one-launch forward's counter workspace: too small, misaligned
+    fneed = ctypes.c_size_t(0)
+    nt3, arr3 = _tiles((1, 2, 2), (1, 4, 4))
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(d), nt3, arr3, 1, ctypes.byref(fneed)) == OK
+    assert _mfwd(lib, d, (nt3, arr3), ws=FAKE, ws_bytes=fneed.value - 4) == WORKSPACE
+    assert _mfwd(lib, d, (nt3, arr3), ws=MISALIGNED, ws_bytes=fneed.value) == ALIGN
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(d), nt3, arr3, 1, None) == INVALID
+    # without inter (inference) the workspace also holds the intermediate outputs
+    assert _mfwd(lib, d, (nt3, arr3), inter=None) == WORKSPACE                      # no workspace at all
+    assert _mfwd(lib, d, (nt3, arr3), inter=None, ws=FAKE, ws_bytes=fneed.value) == WORKSPACE
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(d), nt3, arr3, 0, ctypes.byref(fneed)) == OK
+    assert _mfwd(lib, d, (nt3, arr3), inter=None, ws=FAKE, ws_bytes=fneed.value - 1) == WORKSPACE
     # bf16: a pass whose box row (t_j / t_{j-1} along W) exceeds 128 tokens
     wide = _desc(T=1, H=1, W=512, tT=1, tH=1, tW=1)
     assert _mfwd(lib, wide, _tiles((1, 1, 2), (1, 1, 512))) == UNSUPPORTED
@@ -172,6 +184,16 @@ def test_multi_pass_workspace_size(lib):
     d = _desc(T=4, H=8, W=8)
     nt, arr = _tiles((1, 2, 2), (1, 4, 4))
     got = ctypes.c_size_t(0)
+    # forward: one uint32 counter per (pass 2..k, batch, head), rounded up to 256 bytes
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(d), nt, arr, 1, ctypes.byref(got)) == OK
+    assert got.value == 256
+    big = _desc(B=3, heads=40, T=4, H=8, W=8)
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(big), nt, arr, 1, ctypes.byref(got)) == OK
+    assert got.value == 1024                     # passes 2 and 3 x 120 heads x 4 bytes = 960, rounded up
+    # inference: the outputs of passes 1 and 2 (bf16 [3, 40, 256, 128]) before the counters
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(big), nt, arr, 0, ctypes.byref(got)) == OK
+    assert got.value == 2 * 3 * 40 * 256 * 128 * 2 + 1024
+
     assert lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(d), nt, arr, ctypes.byref(got)) == OK
     rows = 1 * 2 * 256
     # two bf16 upstream gradients, four fp32 accumulators, one fp32 row vector

@@ -105,13 +105,17 @@ def test_k_pass_writes_stay_inside_their_buffers(cuda_ok, grid, tiles, dtype):
     need = ctypes.c_size_t(0)
     assert lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(desc), nt, tarr, ctypes.byref(need)) == 0
     ws = Guarded((need.value,), torch.uint8, dev)
+    fneed = ctypes.c_size_t(0)
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(desc), nt, tarr, 1, ctypes.byref(fneed)) == 0
+    fws = Guarded((fneed.value,), torch.uint8, dev)
     assert lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, tarr, _p(q), _p(k), _p(v), _p(o), _p(inter), _p(lse),
-                                    _stream()) == 0
+                                    _p(fws), fneed.value, _stream()) == 0
     assert lib.squad_attn_multi_bwd(ctypes.byref(desc), nt, tarr, _p(q), _p(k), _p(v), _p(o), _p(inter), _p(lse),
                                     _p(do), _p(dq), _p(dk), _p(dv), _p(ws), need.value, _stream()) == 0
     torch.cuda.synchronize()
     sq.poll_device_error()
-    for name, g in (("o", o), ("inter", inter), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("ws", ws)):
+    for name, g in (("o", o), ("inter", inter), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv), ("ws", ws),
+                    ("fws", fws)):
         assert g.intact(), name
 
 
@@ -139,4 +143,30 @@ def test_inference_forward_writes_stay_inside_their_buffers(cuda_ok, grid, tile,
     assert o.intact() and ws.intact()
     ref, *_ = sq.squad_attn_fwd(q, k, v, grid, tile, save=True)
     sq.poll_device_error()
+    assert torch.equal(o.t, ref)
+
+
+@pytest.mark.parametrize("grid,tiles,dtype", [
+    ((4, 22, 40), [(1, 1, 20), (2, 11, 20)], torch.bfloat16),
+    ((2, 4, 8), [(1, 2, 2), (2, 2, 4)], torch.float32),
+])
+def test_k_pass_inference_writes_stay_inside_their_buffers(cuda_ok, grid, tiles, dtype):
+    # no inter: the intermediate outputs live in the workspace (and leave L2 unwritten on bf16)
+    lib = sq.load_library()
+    inp = random_problem(79, 1, 3, 128 if dtype == torch.bfloat16 else 64, grid, (1, 1, 1), dtype=dtype)
+    dev = torch.device("cuda", 0)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    desc = sq.make_desc(q, grid, tiles[0], None)
+    nt = len(tiles)
+    tarr = (ctypes.c_int * (3 * nt))(*[x for t in tiles for x in t])
+    o = Guarded(q.shape, q.dtype, dev)
+    need = ctypes.c_size_t(0)
+    assert lib.squad_attn_multi_fwd_workspace_size(ctypes.byref(desc), nt, tarr, 0, ctypes.byref(need)) == 0
+    ws = Guarded((need.value,), torch.uint8, dev)
+    assert lib.squad_attn_multi_fwd(ctypes.byref(desc), nt, tarr, _p(q), _p(k), _p(v), _p(o), None, None,
+                                    _p(ws), need.value, _stream()) == 0
+    torch.cuda.synchronize()
+    sq.poll_device_error()
+    assert o.intact() and ws.intact()
+    ref, _, _ = sq.squad_attn_multi_fwd(q, k, v, grid, tiles)
     assert torch.equal(o.t, ref)

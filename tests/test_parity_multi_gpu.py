@@ -166,3 +166,45 @@ def test_packed_passes_are_deterministic(cuda_ok):
     sq.poll_device_error()
     for a, b in zip(first, second):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B,heads,grid,tiles,d", [
+    (1, 1, (2, 8, 16), [(1, 1, 2), (1, 2, 4), (2, 4, 8)], 128),   # one head: no full block
+    (1, 3, (4, 22, 40), [(1, 1, 20), (2, 11, 20)], 128),          # packed passes, heads < 2 lags
+    (2, 3, (2, 8, 16), [(1, 2, 2), (1, 4, 4)], 64),
+    (1, 7, (2, 8, 16), [(1, 1, 2), (1, 2, 2), (1, 4, 8), (2, 8, 8)], 64),   # five passes
+    (2, 5, (2, 16, 64), [(1, 4, 64), (2, 8, 64)], 128),           # 256-token problems: two boxes each
+])
+def test_one_launch_equals_one_launch_per_pass(cuda_ok, B, heads, grid, tiles, d):
+    # the chained launch runs each job exactly as the per-pass launches do: bitwise equal
+    inp = random_problem(61, B, heads, d, grid, (1, 1, 1), dtype=torch.bfloat16)
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    one = sq.squad_attn_multi_fwd(q, k, v, grid, tiles, one_launch=True)
+    per = sq.squad_attn_multi_fwd(q, k, v, grid, tiles, one_launch=False)
+    inf, _, _ = sq.squad_attn_multi_fwd(q, k, v, grid, tiles, save=False)   # intermediates in scratch
+    sq.poll_device_error()
+    for name, a, b in zip(("o", "inter", "lse"), one, per):
+        assert torch.equal(a, b), name
+    assert torch.equal(inf, one[0])
+
+
+def test_one_launch_three_passes_full_size(cuda_ok):
+    # the 27,280-token shape, 24 heads, three passes in one launch: bitwise the per-pass result,
+    # and within the three-pass bf16 budget of the oracle on two heads
+    wl = WORKLOADS["wan5b_fwd"]
+    inp = make_inputs(wl)
+    tiles = [(1, 1, 20), (1, 11, 20)]
+    q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
+    one = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles, one_launch=True)
+    per = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles, one_launch=False)
+    inf, _, _ = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles, save=False)
+    sq.poll_device_error()
+    for name, a, b in zip(("o", "inter", "lse"), one, per):
+        assert torch.equal(a, b), name
+    assert torch.equal(inf, one[0])
+    fmax, fmean, _ = _bf16_tol(3)
+    for h in (5, 23):
+        sel = (slice(0, 1), slice(h, h + 1))
+        ro, _, _, _ = oracle.squad_fwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, tiles)
+        mx, mean = _err(_np(one[0][sel]), ro)
+        assert mx <= fmax and mean <= fmean, (h, mx, mean)

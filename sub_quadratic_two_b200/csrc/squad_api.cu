@@ -53,7 +53,7 @@ struct DeviceState {
   int sms = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
   bool fwd_attr_set[2][2] = {};  // [D=64/128][packed]
-  bool fused_attr_set[2][2] = {};   // [D=64/128][out_f32]
+  bool fused_attr_set[2][2][2] = {};   // [D=64/128][out_f32][packed]
 };
 
 std::mutex g_mu;
@@ -340,12 +340,12 @@ squad_status simt_bwd_t(const Plan& p, const BwdWs& w, uint8_t* ws, const void* 
 
 // ---------------- tensor-core backward (bf16)
 
-template <int D, bool F32>
+template <int D, bool F32, bool PACKED>
 squad_status launch_bwd_fused_t(DeviceState* ds, const CUtensorMap* maps, const sq::BwdFusedArgs& a,
                                 cudaStream_t st) {
   using Lay = sq::BwdFusedLayout<D>;
-  auto kern = sq::squad_bwd_fused_kernel<D, F32>;
-  bool& attr = ds->fused_attr_set[D == 128 ? 1 : 0][F32 ? 1 : 0];
+  auto kern = sq::squad_bwd_fused_kernel<D, F32, PACKED>;
+  bool& attr = ds->fused_attr_set[D == 128 ? 1 : 0][F32 ? 1 : 0][PACKED ? 1 : 0];
   if (!attr) {
     SQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC));
     attr = true;
@@ -402,9 +402,19 @@ squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, c
     if (dq_acc == nullptr) return SQUAD_ERR_INVALID_ARG;
     f.acc_q = dq_acc;
   }
-  squad_status s2 =
-      d == 128 ? (f32_out ? launch_bwd_fused_t<128, true>(ds, maps, f, st) : launch_bwd_fused_t<128, false>(ds, maps, f, st))
-               : (f32_out ? launch_bwd_fused_t<64, true>(ds, maps, f, st) : launch_bwd_fused_t<64, false>(ds, maps, f, st));
+  // packed boxes (problems of at most 64 tokens several to a box) take the masked instance
+  const bool packed = g.pk > 1;
+  squad_status s2;
+  if (d == 128)
+    s2 = f32_out ? (packed ? launch_bwd_fused_t<128, true, true>(ds, maps, f, st)
+                           : launch_bwd_fused_t<128, true, false>(ds, maps, f, st))
+                 : (packed ? launch_bwd_fused_t<128, false, true>(ds, maps, f, st)
+                           : launch_bwd_fused_t<128, false, false>(ds, maps, f, st));
+  else
+    s2 = f32_out ? (packed ? launch_bwd_fused_t<64, true, true>(ds, maps, f, st)
+                           : launch_bwd_fused_t<64, true, false>(ds, maps, f, st))
+                 : (packed ? launch_bwd_fused_t<64, false, true>(ds, maps, f, st)
+                           : launch_bwd_fused_t<64, false, false>(ds, maps, f, st));
   if (s2 != SQUAD_OK || g.nt == 1 || f32_out) return s2;
   const unsigned cblocks = unsigned((n_el / 8 + 255) / 256);
   sq::f32_to_bf16_kernel<<<cblocks, 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), n_el / 8);
@@ -961,7 +971,8 @@ squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int*
   const void* up = dout;
   int acc = 0;  // accumulator holding the sum so far (valid for j < k)
   for (int j = mp.k; j >= 1; --j) {
-    const Geom& g = mp.g[j - 1];
+    // bf16: small problems packed several to a box, as in the forward
+    const Geom& g = bf16 ? mp.gf[j - 1] : mp.g[j - 1];
     const void* val = j == 1 ? v : inter_at(j - 1);
     const void* out = j == mp.k ? o : inter_at(j);
     const float* l = lse + size_t(mp.base.rows) * (j - 1);

@@ -27,6 +27,11 @@
 // nt > 1 each block adds its part into an fp32 buffer with vector reductions
 // (red.global.add.v4.f32) and the host converts that buffer afterwards.
 //
+// Packed geometry (PACKED, problems of at most 64 tokens, several to a box; nt == 1):
+// the softmax-gradient warps zero P and dS between a key row and the query columns of
+// the other problems in the box, and rows past the packed digit's extent are dead on
+// both sides (not read as statistics, not written).
+//
 // Warp roles: warps 0-3 softmax gradient (thread = key row = TMEM lane), warps 4-7
 // epilogue (thread = token row; stores pass through a per-warp transpose patch so that
 // each warp instruction writes whole lines), warp 8 TMA producer, warp 9 MMA issuer.
@@ -298,7 +303,13 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* 
       make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
-template <int D, bool OUT_F32>
+// Packed geometry: whether box row `row` of the box whose first problem is j0 along the
+// packed digit holds a problem (rows past the digit's extent are padding).
+__device__ __forceinline__ bool packed_row_live(const Geom& g, int j0, int row) {
+  return j0 + pack_id(g, row) < g.pk_ext;
+}
+
+template <int D, bool OUT_F32, bool PACKED>
 __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     squad_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -486,16 +497,25 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
+    // packed boxes: the query columns in this key row's problem (the same for every box)
+    uint32_t pmask[4] = {~0u, ~0u, ~0u, ~0u};
+    if (PACKED && g.pk > 1) {
+      const int me = pack_id(g, row);
+#pragma unroll 1
+      for (int j = 0; j < 128; ++j)
+        if (pack_id(g, j) != me) pmask[j >> 5] &= ~(1u << (j & 31));
+    }
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
       const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
-      const int base = problem_base(g, prob);
-      const bool rlive = row < tile_valid_rows(g, kb);
+      int j0 = 0;
+      const int base = problem_base(g, prob, &j0);
+      const bool rlive = row < tile_valid_rows(g, kb) && (!PACKED || g.pk <= 1 || packed_row_live(g, j0, row));
       for (int qb = 0; qb < nt; ++qb, ++t) {
         // per-query statistics of the block's query box: row r publishes column r
         float* vl = vec + (t & 1u) * 256;
-        const bool qlive = row < tile_valid_rows(g, qb);
+        const bool qlive = row < tile_valid_rows(g, qb) && (!PACKED || g.pk <= 1 || packed_row_live(g, j0, row));
         const int tok = qlive ? base + tile_row_offset(g, qb, row) : 0;
         vl[row] = qlive ? args.lse[tok] * log2e : INFINITY;  // query columns past the problem: P = 0
         if (args.Drow != nullptr) {
@@ -551,8 +571,10 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
             float p[4], dsv[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              // key rows past the problem: P = dS = 0 (a select: exp2 of a zero score may overflow)
-              p[u] = rlive ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
+              // key rows past the problem, and in a packed box the query columns of other
+              // problems: P = dS = 0 (a select: exp2 of a zero score may overflow)
+              const bool same = !PACKED || ((pmask[c] >> (e4 + u)) & 1u);
+              p[u] = rlive && same ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
               dsv[u] = p[u] * (__uint_as_float(dp[e4 + u]) - dcol[u]);
             }
             pk[e4 >> 1] = pack_bf16x2(p[0], p[1]);
@@ -588,9 +610,11 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x, ++i) {
       const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
-      const int base = problem_base(g, prob);
+      int j0 = 0;
+      const int base = problem_base(g, prob, &j0);
+      const bool prow = !PACKED || g.pk <= 1 || packed_row_live(g, j0, row);
       for (int qb = 0; qb < nt; ++qb, ++t) {
-        const bool liveq = row < tile_valid_rows(g, qb);
+        const bool liveq = row < tile_valid_rows(g, qb) && prow;
         const EpiRows RQ = epi_rows_of(lane, liveq ? base + tile_row_offset(g, qb, row) : 0, liveq);
         if (!(ok = wwait(&bars[G_DQDONE], t & 1u))) break;
         tc_fence_after();
@@ -603,7 +627,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         mbar_arrive(&bars[G_DQFREE]);
       }
       if (!ok) break;
-      const bool livek = row < tile_valid_rows(g, kb);
+      const bool livek = row < tile_valid_rows(g, kb) && prow;
       const EpiRows RK = epi_rows_of(lane, livek ? base + tile_row_offset(g, kb, row) : 0, livek);
       if (!(ok = wwait(&bars[G_ITEMACC], i & 1u))) break;
       tc_fence_after();

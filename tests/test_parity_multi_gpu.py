@@ -43,6 +43,13 @@ def _err(a, b):
     return float(e.max()), float(e.mean())
 
 
+def _err_scaled(a, b):
+    """max |a - b| / max(1, |b|): the gradient bound at large magnitudes, where the bf16
+    rounding of the result is relative (tests/test_kpass_error_budget.py)."""
+    b = np.asarray(b, np.float64)
+    return float((np.abs(np.asarray(a, np.float64) - b) / np.maximum(1.0, np.abs(b))).max())
+
+
 def _gpu_fwd_bwd(inp, grid, tiles, scale=None):
     q, k, v, do = (t.contiguous().cuda() for t in (inp.q, inp.k, inp.v, inp.do))
     o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, grid, tiles, scale)
@@ -208,3 +215,25 @@ def test_one_launch_three_passes_full_size(cuda_ok):
         ro, _, _, _ = oracle.squad_fwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], wl.grid, tiles)
         mx, mean = _err(_np(one[0][sel]), ro)
         assert mx <= fmax and mean <= fmean, (h, mx, mean)
+
+
+def test_three_passes_backward_full_size(cuda_ok):
+    # the 27,280-token shape, 24 heads, three passes: forward in one launch, backward with the
+    # 20- and 11-token groups packed six and ten to a box; two heads against the oracle
+    # (head 20 has gradients up to 8.8: the bound applies to |err| / max(1, |ref|))
+    wl = WORKLOADS["wan5b_fwd"]
+    inp = make_inputs(wl)
+    tiles = [(1, 1, 20), (1, 11, 20)]
+    g = torch.Generator().manual_seed(97)
+    do = torch.randn(inp.q.shape, generator=g).to(torch.bfloat16)
+    q, k, v, dog = (t.cuda() for t in (inp.q, inp.k, inp.v, do))
+    o, inter, lse = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles)
+    dq, dk, dv = sq.squad_attn_multi_bwd(q, k, v, o, inter, lse, dog, wl.grid, tiles)
+    sq.poll_device_error()
+    _, _, gmax = _bf16_tol(3)
+    for h in (3, 20):
+        sel = (slice(0, 1), slice(h, h + 1))
+        ref = oracle.squad_bwd_multi(inp.q[sel], inp.k[sel], inp.v[sel], do[sel], wl.grid, tiles)
+        for name, a, b in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
+            assert np.isfinite(_np(a[sel])).all(), name
+            assert _err_scaled(_np(a[sel]), b) <= gmax, (h, name)

@@ -42,14 +42,15 @@ METRIC = "SQuad-attn fwd ms & TFLOP/s at 27,280 tokens; % of B200 bf16 TC peak"
 HEADLINE = "wan5b_fwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
-HOST_LEAD_CYCLES = 100_000  # device-side spin after each flush, about 50 us at 1.9 GHz
+HOST_LEAD_CYCLES = 600_000  # device-side spin after each flush, about 300 us at 1.9 GHz
 
 
 def flush_l2(buf):
-    """Evict L2 (write a buffer larger than it), then spin on the device for about 50 us.
+    """Evict L2 (write a buffer larger than it), then spin on the device for about 300 us.
     Both run before the timed region's start event; the spin lets the host enqueue the timed
     call before that event fires, so the events time the device work and not the Python
     call's launch overhead (the end-to-end number covers the host)."""
+    import torch
     buf.zero_()
     torch.cuda._sleep(HOST_LEAD_CYCLES)
 
@@ -76,7 +77,8 @@ def parse_args():
                          "27,280-token shape with B=1 (bf16); no timing")
     ap.add_argument("--profile-kpass", action="store_true",
                     help="profiling driver for three passes over 1x1x20 | 1x11x20 | grid on the 27,280-token "
-                         "shape: two rounds of one inference-form and one training-form launch; no timing")
+                         "shape: two rounds of one inference-form launch, one training-form launch and its "
+                         "backward; no timing")
     ap.add_argument("--profile", action="store_true",
                     help="profiling driver: one warm-up then one measured launch each of the fused forward, the "
                          "local pass alone and the global pass alone; no timing")
@@ -355,7 +357,7 @@ def run_sp(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
                        "grid": list(wl.grid), "tile": list(wl.tile), "useful_flops_per_step": flops,
-                       "l2": "flushed (512 MiB write) before every timed step, then a 50 us device spin outside the timed region",
+                       "l2": "flushed (512 MiB write) before every timed step, then a 300 us device spin outside the timed region",
                        "parallelism": f"sequence-parallel x{world} (frames sharded; two NCCL all-to-alls per step)"},
             "exchange_bytes_per_step_all_ranks": xbytes,
             "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"], "source": peak_src},
@@ -426,9 +428,11 @@ def main():
     if args.profile_kpass:
         tiles3 = [(1, 1, 20), (1, 11, 20)]
         ws3 = torch.empty(sq.multi_fwd_workspace_size(q, wl.grid, tiles3, save=False), device=dev, dtype=torch.uint8)
-        for _ in range(2):  # launch order: inference form, training form (twice)
+        do3 = torch.randn_like(q)
+        for _ in range(2):  # launch order: inference form, training form, its backward (twice)
             sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3, save=False, out=o, workspace=ws3)
-            sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3)
+            mo, minter, mlse = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3)
+            sq.squad_attn_multi_bwd(q, k, v, mo, minter, mlse, do3, wl.grid, tiles3)
             torch.cuda.synchronize()
         sq.poll_device_error()
         print("profile-kpass run done")
@@ -666,7 +670,7 @@ def main():
             "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
                        "grid": list(wl.grid), "tile": list(wl.tile), "w": wl.w, "m": wl.m,
                        "useful_flops_per_step": flops,
-                       "l2": "flushed (512 MiB write) before every timed step, then a 50 us device spin outside the timed region; inputs 503 MB > L2",
+                       "l2": "flushed (512 MiB write) before every timed step, then a 300 us device spin outside the timed region; inputs 503 MB > L2",
                        "parallelism": f"replicas x{world} (independent problems per GPU)"},
             "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
                                   "measured_sustained": value / world / peaks.get("bf16_tflops_sustained", 1),

@@ -191,8 +191,8 @@ squad_status squad_attn_multi_fwd(const squad_desc* desc, int ntiles, const int*
                                   size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace squad_attn_multi_bwd needs: two upstream-gradient
- * tensors of the input dtype, four fp32 [B, heads, n, d] accumulators and one
- * fp32 row vector (each part 256-byte aligned). */
+ * tensors of the input dtype, four fp32 [B, heads, n, d] accumulators and
+ * three fp32 row vectors (each part 256-byte aligned). */
 squad_status squad_attn_multi_bwd_workspace_size(const squad_desc* desc, int ntiles, const int* tiles,
                                                  size_t* bytes);
 

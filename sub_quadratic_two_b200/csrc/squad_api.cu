@@ -422,6 +422,15 @@ squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, c
   return SQUAD_OK;
 }
 
+// D = rowsum(a o b) over bf16 [rows, d] tensors into an fp32 vector.
+squad_status rowdot_bf16(const void* a, const void* b, float* out, long long rows, int d, cudaStream_t st) {
+  const long long threads = rows * (d / 8);
+  sq::rowdot_bf16_kernel<<<unsigned((threads + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), out, rows, d);
+  SQ_CUDA(cudaGetLastError());
+  return SQUAD_OK;
+}
+
 squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws, const void* q, const void* k,
                     const void* v, const void* o, const void* o1, const float* lse1, const float* lse2,
                     const void* dout, void* dq, void* dk, void* dv, int d, cudaStream_t st) {
@@ -429,10 +438,14 @@ squad_status tc_bwd(DeviceState* ds, const Plan& p, const BwdWs& w, uint8_t* ws,
   float* dQ2 = reinterpret_cast<float*>(ws + w.dq2);
   float* dK2 = reinterpret_cast<float*>(ws + w.dk2);
   float* D1 = reinterpret_cast<float*>(ws + w.D1);
+  float* D2 = reinterpret_cast<float*>(ws + w.D2);
   squad_status s;
+  // D2 = rowsum(dout o O) by a bandwidth-bound row-dot pass (in the backward kernel these
+  // loads would sit on each block's critical path)
+  if ((s = rowdot_bf16(dout, o, D2, p.rows, d, st)) != SQUAD_OK) return s;
   // global pass: values O1, output O, upstream dout -> dQ2, dK2 (fp32), dO1 and the
-  // local pass's D1 = rowsum(dO1 o O1); its own D is computed in the kernel
-  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, nullptr, D1, nullptr, nullptr, dQ2, nullptr, dK2, dO1,
+  // local pass's D1 = rowsum(dO1 o O1)
+  s = tc_pass_bwd(ds, p, d, p.g2, q, k, o1, o, dout, lse2, D2, D1, nullptr, nullptr, dQ2, nullptr, dK2, dO1,
                   true, st);
   if (s != SQUAD_OK) return s;
   // local pass: values V, output O1, upstream dO1 -> dq = dq1 + dQ2, dk = dk1 + dK2, dv
@@ -830,7 +843,7 @@ squad_status launch_fwd_multi(DeviceState* ds, int d, const MultiPlan& mp, const
 // fp32 dK accumulators used in turn (the pass reads one and writes the other), one fp32
 // row vector.
 struct MultiWs {
-  size_t up[2], dq[2], dk[2], drow, total;
+  size_t up[2], dq[2], dk[2], drow, dvec[2], total;
 };
 
 MultiWs multi_workspace(const MultiPlan& mp, const squad_desc* d) {
@@ -842,6 +855,7 @@ MultiWs multi_workspace(const MultiPlan& mp, const squad_desc* d) {
   for (int i = 0; i < 2; ++i) { w.dk[i] = off; off += align256(big * 4); }
   w.drow = off;
   off += align256(size_t(mp.base.rows) * 4);
+  for (int i = 0; i < 2; ++i) { w.dvec[i] = off; off += align256(size_t(mp.base.rows) * 4); }
   w.total = off;
   return w;
 }
@@ -970,6 +984,11 @@ squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int*
   // the first pass writes the final dq, dk, dv.
   const void* up = dout;
   int acc = 0;  // accumulator holding the sum so far (valid for j < k)
+  // bf16: D of pass k = rowsum(dout o o) by a row-dot pass; pass j writes the D of pass j-1
+  // (rowsum(dVal o Val) of its own results) into the other vector
+  if (bf16 && (s = rowdot_bf16(dout, o, reinterpret_cast<float*>(ws + w.dvec[mp.k & 1]), mp.base.rows, desc->d,
+                               st)) != SQUAD_OK)
+    return s;
   for (int j = mp.k; j >= 1; --j) {
     // bf16: small problems packed several to a box, as in the forward
     const Geom& g = bf16 ? mp.gf[j - 1] : mp.g[j - 1];
@@ -985,7 +1004,9 @@ squad_status squad_attn_multi_bwd(const squad_desc* desc, int ntiles, const int*
       // the last step (j = 1) writes bf16 and, for multi-box problems, adds its dQ parts
       // into the fp32 sum before the conversion
       float* q_acc = j == 1 ? const_cast<float*>(q_add) : nullptr;
-      s = tc_pass_bwd(ds, mp.base, desc->d, g, q, k, val, out, up, l, nullptr, nullptr, q_add, q_acc, q_out,
+      const float* drow = reinterpret_cast<const float*>(ws + w.dvec[j & 1]);
+      float* d_next = j > 1 ? reinterpret_cast<float*>(ws + w.dvec[(j - 1) & 1]) : nullptr;
+      s = tc_pass_bwd(ds, mp.base, desc->d, g, q, k, val, out, up, l, drow, d_next, q_add, q_acc, q_out,
                       k_add, k_out, static_cast<__nv_bfloat16*>(dval), j > 1, st);
     } else {
       s = simt_pass_bwd_f32_any(desc->d, g, mp.base.rows, static_cast<const float*>(q),

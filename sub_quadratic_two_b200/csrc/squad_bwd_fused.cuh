@@ -32,9 +32,10 @@
 // the other problems in the box, and rows past the packed digit's extent are dead on
 // both sides (not read as statistics, not written).
 //
-// Warp roles: warps 0-3 softmax gradient (thread = key row = TMEM lane), warps 4-7
-// epilogue (thread = token row; stores pass through a per-warp transpose patch so that
-// each warp instruction writes whole lines), warp 8 TMA producer, warp 9 MMA issuer.
+// Warp roles: warps 0-3 softmax gradient (thread = key row = TMEM lane), then the drain of
+// the block's dQ part (thread = query row); warps 4-7 epilogue, the drain of dVal and dK
+// (thread = token row); warp 8 TMA producer, warp 9 MMA issuer. Drains pass through
+// per-warp transpose patches so that each warp instruction writes whole lines.
 // Input tiles live in a pool of five slots handed out in the order they are freed, so
 // the next block's Q (and, at an item boundary, K) load while the current block's
 // gradients are still accumulating. Every wait is bounded.
@@ -76,7 +77,8 @@ struct BwdFusedLayout {
   static constexpr int SLOT_OFF = 0;
   static constexpr int DS_OFF = NSLOT * TILE;           // dS^T: 128 key rows x 128 query columns, bf16
   static constexpr int XP_OFF = DS_OFF + 128 * 128 * 2;  // 4 epilogue warps x (32 rows x 128 B)
-  static constexpr int VEC_OFF = XP_OFF + 4 * 4096;      // 2 buffers x (lse*log2e[128], D[128])
+  static constexpr int XPS_OFF = XP_OFF + 4 * 4096;      // 4 softmax warps x (16 rows x 128 B)
+  static constexpr int VEC_OFF = XPS_OFF + 4 * 2048;     // 2 buffers x (lse*log2e[128], D[128])
   static constexpr int BAR_OFF = VEC_OFF + 2 * 256 * 4;
   static constexpr int NBAR = 20;
   static constexpr int BYTES = BAR_OFF + NBAR * 8 + 16;
@@ -243,6 +245,67 @@ __device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, c
   }
 }
 
+// The same drain through a patch of 16 rows (the softmax warps' patches are half the size
+// of the epilogue warps'): per 32-column chunk, lanes 0-15 and then lanes 16-31 write their
+// rows, and each round is written back four rows per instruction (lane l: patch row
+// 4i + l/8, 16-byte chunk l%8).
+template <int D, int KIND>
+__device__ __forceinline__ void epi_acc16(uint32_t taddr, uint32_t xp, int lane, int my_tok, bool my_live,
+                                          float scale, const float* add, void* out) {
+  const int pr = lane >> 3, lc = lane & 7;
+  const uint32_t live = __ballot_sync(0xffffffffu, my_live);
+  int tok[2][4];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tok[r][i] = __shfl_sync(0xffffffffu, my_tok, 16 * r + 4 * i + pr);
+  const int prow = lane & 15;
+#pragma unroll 1
+  for (int ch = 0; ch < D / 32; ++ch) {
+    float4 a[2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[r][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (add != nullptr && ((live >> (16 * r + 4 * i + pr)) & 1u))
+          a[r][i] = __ldg(reinterpret_cast<const float4*>(add + size_t(tok[r][i]) * D + ch * 32 + lc * 4));
+      }
+    uint32_t v[32];
+    tmem_ld32(taddr + ch * 32, v);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if ((lane >> 4) == r) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(xp + prow * 128 + ((c ^ (prow & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * c]) * scale),
+                       __float_as_uint(__uint_as_float(v[4 * c + 1]) * scale),
+                       __float_as_uint(__uint_as_float(v[4 * c + 2]) * scale),
+                       __float_as_uint(__uint_as_float(v[4 * c + 3]) * scale));
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int q = 4 * i + pr;
+        const uint4 x = ld_shared_v4(xp + q * 128 + ((lc ^ (q & 7)) << 4));
+        if ((live >> (16 * r + q)) & 1u) {
+          const float f0 = __uint_as_float(x.x) + a[r][i].x, f1 = __uint_as_float(x.y) + a[r][i].y;
+          const float f2 = __uint_as_float(x.z) + a[r][i].z, f3 = __uint_as_float(x.w) + a[r][i].w;
+          const size_t e = size_t(tok[r][i]) * D + ch * 32 + lc * 4;
+          if (KIND == EPI_F32)
+            *reinterpret_cast<float4*>(static_cast<float*>(out) + e) = make_float4(f0, f1, f2, f3);
+          else if (KIND == EPI_BF16)
+            *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out) + e) =
+                make_uint2(pack_bf16x2(f0, f1), pack_bf16x2(f2, f3));
+          else
+            red_add_v4(static_cast<float*>(out) + e, f0, f1, f2, f3);
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
 // Drain one fp32 accumulator as bf16 rows (no scale), 64 columns per round; with
 // d_next, also rowsum(value o val) of the written (bf16) values, one float per row.
 template <int D>
@@ -291,6 +354,25 @@ __device__ __forceinline__ void epi_acc_bf16(uint32_t taddr, uint32_t xp, int la
       if (lc == 0 && ((R.live >> (4 * i + lr)) & 1u)) d_next[R.tok[i]] = v;
     }
   }
+}
+
+// D_t = rowsum(a_t o b_t) of bf16 rows (d a multiple of 8, at most 256): d/8 threads per
+// row, one 16-byte chunk of each operand per thread, a shuffle sum over the row's lanes.
+// Coalesced and HBM-bound; it gives the first backward launch its D as a vector.
+__global__ void rowdot_bf16_kernel(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b,
+                                   float* __restrict__ out, long long rows, int d) {
+  const int per = d / 8;  // lanes per row: a power of two dividing 32 (d = 64 or 128)
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = gid / per;
+  const int c = int(gid - row * per);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(a + row * d) + c);
+    const uint4 y = __ldg(reinterpret_cast<const uint4*>(b + row * d) + c);
+    acc = dot8_bf16(x, y, 0.f);
+  }
+  for (int off = per >> 1; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && c == 0) out[row] = acc;
 }
 
 // dq = bf16(acc), 8 elements per thread (rows * d is a multiple of 8)
@@ -492,6 +574,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     const uint32_t lane_sel = uint32_t(warp * 32) << 16;
     const uint32_t tS = tmem + lane_sel + Lay::TM_S, tDP = tmem + lane_sel + Lay::TM_DP;
     const uint32_t ds_row = sbase + Lay::DS_OFF + row * 128;
+    const uint32_t xps = sbase + Lay::XPS_OFF + warp * 2048;
     const float c2 = args.scale_log2;
     const float log2e = 1.4426950408889634f;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
@@ -595,6 +678,17 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         fence_async_smem();  // the dS^T tile is read by the tensor core
         tc_fence_before();
         mbar_arrive(&bars[G_PFULL]);
+        // the block's dQ part (TMEM lane = query row): drained here while the epilogue warps
+        // drain dVal and dK, so the next block's dP^T, which reuses its columns, is not
+        // queued behind the item's other accumulators
+        if (!(ok = wwait(&bars[G_DQDONE], t & 1u))) break;
+        tc_fence_after();
+        if (nt > 1)
+          epi_acc16<D, EPI_RED>(tDP, xps, lane, tok, qlive, args.scale, nullptr, args.acc_q);
+        else
+          epi_acc16<D, OUT_F32 ? EPI_F32 : EPI_BF16>(tDP, xps, lane, tok, qlive, args.scale, args.add_q, args.out_q);
+        tc_fence_before();
+        mbar_arrive(&bars[G_DQFREE]);
       }
     }
   } else {
@@ -606,27 +700,13 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
     };
-    uint32_t i = 0, t = 0;
+    uint32_t i = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x, ++i) {
       const int prob = fdiv(item, g.f_nt), kb = item - prob * nt;
       int j0 = 0;
       const int base = problem_base(g, prob, &j0);
       const bool prow = !PACKED || g.pk <= 1 || packed_row_live(g, j0, row);
-      for (int qb = 0; qb < nt; ++qb, ++t) {
-        const bool liveq = row < tile_valid_rows(g, qb) && prow;
-        const EpiRows RQ = epi_rows_of(lane, liveq ? base + tile_row_offset(g, qb, row) : 0, liveq);
-        if (!(ok = wwait(&bars[G_DQDONE], t & 1u))) break;
-        tc_fence_after();
-        const uint32_t tq = tmem + lane_sel + Lay::TM_DP;
-        if (nt > 1)
-          epi_acc<D, EPI_RED>(tq, xp, lane, RQ, args.scale, nullptr, args.acc_q);
-        else
-          epi_acc<D, OUT_F32 ? EPI_F32 : EPI_BF16>(tq, xp, lane, RQ, args.scale, args.add_q, args.out_q);
-        tc_fence_before();
-        mbar_arrive(&bars[G_DQFREE]);
-      }
-      if (!ok) break;
       const bool livek = row < tile_valid_rows(g, kb) && prow;
       const EpiRows RK = epi_rows_of(lane, livek ? base + tile_row_offset(g, kb, row) : 0, livek);
       if (!(ok = wwait(&bars[G_ITEMACC], i & 1u))) break;

@@ -196,5 +196,5 @@ def test_multi_pass_workspace_size(lib):
 
     assert lib.squad_attn_multi_bwd_workspace_size(ctypes.byref(d), nt, arr, ctypes.byref(got)) == OK
     rows = 1 * 2 * 256
-    # two bf16 upstream gradients, four fp32 accumulators, one fp32 row vector
-    assert got.value == 2 * rows * 128 * 2 + 4 * rows * 128 * 4 + rows * 4
+    # two bf16 upstream gradients, four fp32 accumulators, three fp32 row vectors
+    assert got.value == 2 * rows * 128 * 2 + 4 * rows * 128 * 4 + 3 * rows * 4

@@ -376,9 +376,8 @@ squad_status tc_pass_bwd(DeviceState* ds, const Plan& p, int d, const Geom& g, c
   f.scale = p.scale;
   f.scale_log2 = p.scale * 1.4426950408889634f;
   f.lse = lse;
+  if (Drow == nullptr) return SQUAD_ERR_INVALID_ARG;
   f.Drow = Drow;
-  f.out = static_cast<const __nv_bfloat16*>(out);
-  f.dout = static_cast<const __nv_bfloat16*>(dout);
   f.val = static_cast<const __nv_bfloat16*>(val);
   f.d_next = d_next;
   f.add_k = dk_add;

@@ -7,10 +7,9 @@
 // global pass). Its gradient is the textbook one:
 //   P = exp(s*Q K^T - lse),  dP = dO Val^T,  D = rowsum(dO o O),  dS = P o (dP - D)
 //   dVal = P^T dO,  dK = s * dS^T Q,  dQ = s * dS K.
-// D of a query row is read from a vector or computed by the softmax warps from dO and
-// O rows (four rows per load instruction). The epilogue can also produce the D of the
-// pass that made Val: rowsum(dVal o Val) over the rows it writes (the global pass
-// gives the local pass its D this way).
+// D of a query row is read from a vector (a row-dot pass makes it for the first backward
+// launch). The epilogue can also produce the D of the pass that made Val: rowsum(dVal o
+// Val) over the rows it writes (the global pass gives the local pass its D this way).
 // A problem of L tokens is cut into nt boxes of at most 128 rows. A CTA item is
 // (problem, key box kb): K_kb and Val_kb stay, the query boxes (Q_qb, dO_qb) stream,
 // and every (qb, kb) block is done once, with five GEMMs and no recomputation:
@@ -53,9 +52,7 @@ struct BwdFusedArgs {
   float scale;             // softmax scale
   float scale_log2;        // scale * log2(e)
   const float* lse;        // [rows] natural-log LSE of this pass
-  const float* Drow;          // [rows] D = rowsum(dO o O) of this pass, or nullptr: computed here
-  const __nv_bfloat16* out;   // [rows, D] output of this pass (read when Drow == nullptr)
-  const __nv_bfloat16* dout;  // [rows, D] its upstream gradient (read when Drow == nullptr)
+  const float* Drow;          // [rows] D = rowsum(dO o O) of this pass
   const __nv_bfloat16* val;   // [rows, D] values of this pass (read when d_next != nullptr)
   float* d_next;              // [rows] rowsum(dVal o Val), the D of the pass that produced Val, or nullptr
   const float* add_q;      // nt == 1: fp32 [rows, D] added to dQ, or nullptr
@@ -588,6 +585,23 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
       for (int j = 0; j < 128; ++j)
         if (pack_id(g, j) != me) pmask[j >> 5] &= ~(1u << (j & 31));
     }
+    // the statistics (lse, D) of this thread's query row in a block, read one block ahead so
+    // that their latency overlaps the previous block's dQ drain
+    auto stats_of = [&](int item, int qb, float& lse_l2, float& dv) {
+      lse_l2 = INFINITY;  // query columns past the problem: P = 0
+      dv = 0.f;
+      if (item >= args.total_items) return;
+      const int prob = fdiv(item, g.f_nt);
+      int j0 = 0;
+      const int base = problem_base(g, prob, &j0);
+      if (row < tile_valid_rows(g, qb) && (!PACKED || g.pk <= 1 || packed_row_live(g, j0, row))) {
+        const int tk = base + tile_row_offset(g, qb, row);
+        lse_l2 = __ldg(args.lse + tk) * log2e;
+        dv = __ldg(args.Drow + tk);
+      }
+    };
+    float nx_lse, nx_d;
+    stats_of(blockIdx.x, 0, nx_lse, nx_d);
     uint32_t t = 0;
     bool ok = true;
     for (int item = blockIdx.x; ok && item < args.total_items; item += gridDim.x) {
@@ -600,41 +614,8 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         float* vl = vec + (t & 1u) * 256;
         const bool qlive = row < tile_valid_rows(g, qb) && (!PACKED || g.pk <= 1 || packed_row_live(g, j0, row));
         const int tok = qlive ? base + tile_row_offset(g, qb, row) : 0;
-        vl[row] = qlive ? args.lse[tok] * log2e : INFINITY;  // query columns past the problem: P = 0
-        if (args.Drow != nullptr) {
-          vl[128 + row] = qlive ? args.Drow[tok] : 0.f;
-        } else {
-          // D of the warp's 32 rows: lane l takes rows 4i + l/8, 16-byte chunks l%8 (+8), so
-          // each load instruction reads four whole 128-byte lines; eight lanes sum a row
-          const int lr = lane >> 3, lc = lane & 7;
-          const uint32_t qmask = __ballot_sync(0xffffffffu, qlive);
-#pragma unroll
-          for (int i0 = 0; i0 < 8; i0 += 4) {
-            float part[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int r = 4 * (i0 + u) + lr;
-              const size_t rt = size_t(__shfl_sync(0xffffffffu, tok, r)) * D;
-              part[u] = 0.f;
-              if ((qmask >> r) & 1u) {
-#pragma unroll
-                for (int j = 0; j < D / 64; ++j) {
-                  const uint4 x = __ldg(reinterpret_cast<const uint4*>(args.dout + rt + j * 64 + lc * 8));
-                  const uint4 y = __ldg(reinterpret_cast<const uint4*>(args.out + rt + j * 64 + lc * 8));
-                  part[u] = dot8_bf16(x, y, part[u]);
-                }
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float v = part[u];
-              v += __shfl_xor_sync(0xffffffffu, v, 1);
-              v += __shfl_xor_sync(0xffffffffu, v, 2);
-              v += __shfl_xor_sync(0xffffffffu, v, 4);
-              if (lc == 0) vl[128 + warp * 32 + 4 * (i0 + u) + lr] = v;
-            }
-          }
-        }
+        vl[row] = nx_lse;
+        vl[128 + row] = nx_d;
         mbar_arrive(&bars[G_VEC]);
         if (!(ok = wwait(&bars[G_VEC], t & 1u))) break;
         if (!(ok = wwait(&bars[G_SFULL], t & 1u))) break;
@@ -678,6 +659,10 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         fence_async_smem();  // the dS^T tile is read by the tensor core
         tc_fence_before();
         mbar_arrive(&bars[G_PFULL]);
+        if (qb + 1 < nt)
+          stats_of(item, qb + 1, nx_lse, nx_d);
+        else
+          stats_of(item + int(gridDim.x), 0, nx_lse, nx_d);
         // the block's dQ part (TMEM lane = query row): drained here while the epilogue warps
         // drain dVal and dK, so the next block's dP^T, which reuses its columns, is not
         // queued behind the item's other accumulators

@@ -622,6 +622,8 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
+          // this chunk's 32 query columns of the packed-box mask (selected, not indexed)
+          const uint32_t pm = c == 0 ? pmask[0] : c == 1 ? pmask[1] : c == 2 ? pmask[2] : pmask[3];
           uint32_t s[32], dp[32];
           tmem_ld32(tS + c * 32, s);
           tmem_ld32(tDP + c * 32, dp);
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
             for (int u = 0; u < 4; ++u) {
               // key rows past the problem, and in a packed box the query columns of other
               // problems: P = dS = 0 (a select: exp2 of a zero score may overflow)
-              const bool same = !PACKED || ((pmask[c] >> (e4 + u)) & 1u);
+              const bool same = !PACKED || ((pm >> (e4 + u)) & 1u);
               p[u] = rlive && same ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
               dsv[u] = p[u] * (__uint_as_float(dp[e4 + u]) - dcol[u]);
             }

@@ -42,17 +42,11 @@ METRIC = "SQuad-attn fwd ms & TFLOP/s at 27,280 tokens; % of B200 bf16 TC peak"
 HEADLINE = "wan5b_fwd"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
-HOST_LEAD_CYCLES = 600_000  # device-side spin after each flush, about 300 us at 1.9 GHz
 
 
 def flush_l2(buf):
-    """Evict L2 (write a buffer larger than it), then spin on the device for about 300 us.
-    Both run before the timed region's start event; the spin lets the host enqueue the timed
-    call before that event fires, so the events time the device work and not the Python
-    call's launch overhead (the end-to-end number covers the host)."""
-    import torch
+    """Evict L2 before a timed step: write a buffer larger than it (512 MiB; L2 is 126 MB)."""
     buf.zero_()
-    torch.cuda._sleep(HOST_LEAD_CYCLES)
 
 
 def parse_args():
@@ -357,7 +351,7 @@ def run_sp(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
                        "grid": list(wl.grid), "tile": list(wl.tile), "useful_flops_per_step": flops,
-                       "l2": "flushed (512 MiB write) before every timed step, then a 300 us device spin outside the timed region",
+                       "l2": "flushed (512 MiB write) before every timed step",
                        "parallelism": f"sequence-parallel x{world} (frames sharded; two NCCL all-to-alls per step)"},
             "exchange_bytes_per_step_all_ranks": xbytes,
             "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"], "source": peak_src},
@@ -670,7 +664,7 @@ def main():
             "config": {"workload": wl.name, "B": wl.B, "heads": wl.heads, "n": wl.n, "d": wl.d,
                        "grid": list(wl.grid), "tile": list(wl.tile), "w": wl.w, "m": wl.m,
                        "useful_flops_per_step": flops,
-                       "l2": "flushed (512 MiB write) before every timed step, then a 300 us device spin outside the timed region; inputs 503 MB > L2",
+                       "l2": "flushed (512 MiB write) before every timed step; inputs 503 MB > L2",
                        "parallelism": f"replicas x{world} (independent problems per GPU)"},
             "frac_of_bf16_peak": {"measured_burst": value / world / peaks["bf16_tflops"],
                                   "measured_sustained": value / world / peaks.get("bf16_tflops_sustained", 1),

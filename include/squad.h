@@ -94,6 +94,24 @@ squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k
                             void* o1, float* lse1, float* lse2, void* workspace, size_t workspace_bytes,
                             void* stream);
 
+/* Forward from host memory. q, k, v and o are HOST pointers ([B, heads, n, d]
+ * of the descriptor's dtype; pinned memory for the copies to overlap, pageable
+ * memory works but serialises). The (batch, head) slices are independent, so
+ * the call runs on chunks of slices_per_chunk slices: the copy of chunk i+1 to
+ * the device (on stream_in), the forward of chunk i (on stream, as
+ * squad_attn_fwd without o1) and the copy of chunk i-1 back (on stream_out)
+ * overlap. Results are those of squad_attn_fwd, bitwise. The call is ordered
+ * after the work already on `stream`, and o is complete once `stream` has been
+ * synchronised (all three streams join it). The three streams must differ.
+ * workspace: device, 16-byte aligned, at least
+ * squad_attn_fwd_host_workspace_size bytes (two sets of chunk buffers and the
+ * chunk forward's workspace), owned by the caller, not shared with a call in
+ * flight. Events are created and released inside the call. */
+squad_status squad_attn_fwd_host_workspace_size(const squad_desc* desc, int slices_per_chunk, size_t* bytes);
+squad_status squad_attn_fwd_host(const squad_desc* desc, const void* q, const void* k, const void* v, void* o,
+                                 int slices_per_chunk, void* workspace, size_t workspace_bytes,
+                                 void* stream, void* stream_in, void* stream_out);
+
 /* One pass of the forward, for callers that compose or time the passes on
  * their own. stage 1 (local pass): out = per-window attention with values
  * `val` = v. stage 2 (global pass): out = per-group attention with values

@@ -23,7 +23,7 @@ __all__ = [
     "SquadError", "attention", "squad_attn_fwd", "squad_attn_bwd", "workspace_size",
     "poll_device_error", "library_path", "load_library", "SQUAD_F32", "SQUAD_BF16", "squad_attn_fwd_pass",
     "plan_info", "make_desc", "attention_multi", "squad_attn_multi_fwd", "squad_attn_multi_bwd",
-    "multi_fwd_workspace_size",
+    "multi_fwd_workspace_size", "attention_host",
     "tmap_cache_stats",
 ]
 
@@ -71,6 +71,8 @@ def load_library():
         lib.squad_attn_fwd.argtypes = [dp, vp, vp, vp, vp, vp, fp, fp, vp, sz, vp]
         lib.squad_attn_bwd.argtypes = [dp, vp, vp, vp, vp, vp, fp, fp, vp, vp, vp, vp, vp, sz, vp]
         lib.squad_attn_fwd_pass.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, fp, vp]
+        lib.squad_attn_fwd_host_workspace_size.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+        lib.squad_attn_fwd_host.argtypes = [dp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp, vp, vp]
         lib.squad_plan_info.argtypes = [dp, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
         ip = ctypes.POINTER(ctypes.c_int)
         lib.squad_attn_multi_fwd_workspace_size.argtypes = [dp, ctypes.c_int, ip, ctypes.c_int,
@@ -85,7 +87,8 @@ def load_library():
         lib.squad_strerror.argtypes = [ctypes.c_int]
         lib.squad_strerror.restype = ctypes.c_char_p
         for f in ("squad_attn_workspace_size", "squad_attn_fwd", "squad_attn_bwd", "squad_poll_device_error",
-                  "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_multi_fwd_workspace_size", "squad_attn_multi_fwd",
+                  "squad_attn_fwd_pass", "squad_plan_info", "squad_attn_fwd_host_workspace_size",
+                  "squad_attn_fwd_host", "squad_attn_multi_fwd_workspace_size", "squad_attn_multi_fwd",
                   "squad_attn_multi_bwd_workspace_size", "squad_attn_multi_bwd",
                   "squad_last_cuda_error", "squad_version", "squad_tmap_cache_stats"):
             getattr(lib, f).restype = ctypes.c_int
@@ -280,6 +283,53 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid: Tuple[int
               tile: Tuple[int, int, int], scale: Optional[float] = None) -> torch.Tensor:
     """SQuad-Attention of [B, heads, T*H*W, d] CUDA tensors (float32 or bfloat16), differentiable."""
     return _SquadAttention.apply(q, k, v, tuple(grid), tuple(tile), scale)
+
+
+_side_streams = {}
+
+
+def attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, grid, tile, scale: Optional[float] = None,
+                   out: Optional[torch.Tensor] = None, slices_per_chunk: int = 4,
+                   device: Optional[torch.device] = None, synchronize: bool = True) -> torch.Tensor:
+    """SQuad-Attention forward of HOST tensors [B, heads, n, d] through squad_attn_fwd_host.
+
+    The copies to and from the device overlap the forward, chunk by chunk of
+    (batch, head) slices (pinned host tensors for the overlap). Returns the
+    output as a host tensor (``out``, pinned, when not given). With
+    synchronize=False the call returns once everything is enqueued on the
+    device's current stream; ``out`` is complete after that stream synchronises.
+    """
+    lib = load_library()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous 4-D host tensor")
+        if t.shape != q.shape or t.dtype != q.dtype:
+            raise ValueError("q, k and v must have the same shape and dtype")
+    desc = make_desc(q, grid, tile, scale)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    elif out.is_cuda or not out.is_contiguous() or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must be a contiguous host tensor of q's shape and dtype")
+    nb = ctypes.c_size_t(0)
+    _check(lib.squad_attn_fwd_host_workspace_size(ctypes.byref(desc), int(slices_per_chunk), ctypes.byref(nb)),
+           "squad_attn_fwd_host_workspace_size")
+    with torch.cuda.device(dev):
+        ws = torch.empty(int(nb.value), device=dev, dtype=torch.uint8)
+        if dev.index not in _side_streams:
+            _side_streams[dev.index] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+        s_in, s_out = _side_streams[dev.index]
+        cur = torch.cuda.current_stream(dev)
+        _check(lib.squad_attn_fwd_host(ctypes.byref(desc), ctypes.c_void_p(q.data_ptr()),
+                                       ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+                                       ctypes.c_void_p(out.data_ptr()), int(slices_per_chunk), _ptr(ws), int(nb.value),
+                                       ctypes.c_void_p(cur.cuda_stream), ctypes.c_void_p(s_in.cuda_stream),
+                                       ctypes.c_void_p(s_out.cuda_stream)), "squad_attn_fwd_host")
+        ws.record_stream(s_in)
+        ws.record_stream(s_out)
+        if synchronize:
+            cur.synchronize()
+    return out
 
 
 def squad_attn_fwd_noalloc(q, k, v, grid, tile, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,

@@ -547,6 +547,114 @@ squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k
   return simt_fwd<float>(p.g2, q, k, o1buf, o, lse2, d, p.scale, st);
 }
 
+// ---- forward from host memory, copies overlapped with compute
+// The (batch, head) slices are independent problems, so the forward runs on chunks of
+// slices: the copy of chunk i+1 in, the forward of chunk i and the copy of chunk i-1 out
+// proceed on three streams at once. Device buffers: two sets (q, k, v, o of one chunk)
+// used in turn, then the fused forward's workspace for one chunk.
+namespace {
+
+struct HostFwdWs {
+  size_t set_bytes, chunk_bytes, fwd_ws, total;
+};
+
+HostFwdWs host_fwd_workspace(const squad_desc* d, const Plan& p, int chunk) {
+  squad_desc dc = *d;
+  dc.B = 1;
+  dc.heads = chunk;
+  Plan pc;
+  HostFwdWs w{};
+  w.chunk_bytes = size_t(chunk) * (p.rows / (long long)(d->B * d->heads)) * d->d * p.elem;
+  w.set_bytes = 4 * align256(w.chunk_bytes);
+  w.fwd_ws = make_plan(&dc, &pc) == SQUAD_OK ? fwd_workspace(pc, &dc) : 0;
+  w.total = 2 * w.set_bytes + w.fwd_ws;
+  return w;
+}
+
+struct EventSet {  // events of one call, released when the call has enqueued everything
+  cudaEvent_t e[7] = {};
+  int n = 0;
+  ~EventSet() {
+    for (int i = 0; i < n; ++i) cudaEventDestroy(e[i]);
+  }
+};
+
+}  // namespace
+
+squad_status squad_attn_fwd_host_workspace_size(const squad_desc* desc, int slices_per_chunk, size_t* bytes) {
+  if (bytes == nullptr) return SQUAD_ERR_INVALID_ARG;
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (slices_per_chunk < 1) return SQUAD_ERR_INVALID_ARG;
+  const int S = desc->B * desc->heads;
+  const int chunk = slices_per_chunk < S ? slices_per_chunk : S;
+  *bytes = host_fwd_workspace(desc, p, chunk).total;
+  return SQUAD_OK;
+}
+
+squad_status squad_attn_fwd_host(const squad_desc* desc, const void* q, const void* k, const void* v, void* o,
+                                 int slices_per_chunk, void* workspace, size_t workspace_bytes,
+                                 void* stream, void* stream_in, void* stream_out) {
+  Plan p;
+  squad_status s = make_plan(desc, &p);
+  if (s != SQUAD_OK) return s;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || slices_per_chunk < 1)
+    return SQUAD_ERR_INVALID_ARG;
+  if (stream_in == nullptr || stream_out == nullptr || stream_in == stream_out || stream_in == stream ||
+      stream_out == stream)
+    return SQUAD_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return SQUAD_ERR_ALIGN;
+  const int S = desc->B * desc->heads;
+  const int chunk = slices_per_chunk < S ? slices_per_chunk : S;
+  const HostFwdWs w = host_fwd_workspace(desc, p, chunk);
+  if (workspace == nullptr || workspace_bytes < w.total) return SQUAD_ERR_WORKSPACE;
+  cudaStream_t sc = static_cast<cudaStream_t>(stream), si = static_cast<cudaStream_t>(stream_in),
+               so = static_cast<cudaStream_t>(stream_out);
+  const size_t slice_bytes = w.chunk_bytes / size_t(chunk);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto buf = [&](int set, int which) { return ws + size_t(set) * w.set_bytes + size_t(which) * align256(w.chunk_bytes); };
+  uint8_t* fws = ws + 2 * w.set_bytes;
+  EventSet ev;  // [0] entry, [1..2] copied in, [3..4] computed, [5..6] copied out (per buffer set)
+  for (; ev.n < 7; ++ev.n) SQ_CUDA(cudaEventCreateWithFlags(&ev.e[ev.n], cudaEventDisableTiming));
+  // ordered after the work already on `stream`
+  SQ_CUDA(cudaEventRecord(ev.e[0], sc));
+  SQ_CUDA(cudaStreamWaitEvent(si, ev.e[0], 0));
+  SQ_CUDA(cudaStreamWaitEvent(so, ev.e[0], 0));
+  const uint8_t* hq = static_cast<const uint8_t*>(q);
+  const uint8_t* hk = static_cast<const uint8_t*>(k);
+  const uint8_t* hv = static_cast<const uint8_t*>(v);
+  uint8_t* ho = static_cast<uint8_t*>(o);
+  for (int c0 = 0, i = 0; c0 < S; c0 += chunk, ++i) {
+    const int cs = S - c0 < chunk ? S - c0 : chunk;
+    const int b = i & 1;
+    const size_t off = size_t(c0) * slice_bytes, nb = size_t(cs) * slice_bytes;
+    // set b was last read by the forward of chunk i-2 (inputs) and the copy out of chunk i-2 (output)
+    if (i >= 2) SQ_CUDA(cudaStreamWaitEvent(si, ev.e[3 + b], 0));
+    SQ_CUDA(cudaMemcpyAsync(buf(b, 0), hq + off, nb, cudaMemcpyHostToDevice, si));
+    SQ_CUDA(cudaMemcpyAsync(buf(b, 1), hk + off, nb, cudaMemcpyHostToDevice, si));
+    SQ_CUDA(cudaMemcpyAsync(buf(b, 2), hv + off, nb, cudaMemcpyHostToDevice, si));
+    SQ_CUDA(cudaEventRecord(ev.e[1 + b], si));
+    SQ_CUDA(cudaStreamWaitEvent(sc, ev.e[1 + b], 0));
+    if (i >= 2) SQ_CUDA(cudaStreamWaitEvent(sc, ev.e[5 + b], 0));
+    squad_desc dc = *desc;
+    dc.B = 1;
+    dc.heads = cs;
+    if ((s = squad_attn_fwd(&dc, buf(b, 0), buf(b, 1), buf(b, 2), buf(b, 3), nullptr, nullptr, nullptr, fws, w.fwd_ws,
+                            sc)) != SQUAD_OK)
+      return s;
+    SQ_CUDA(cudaEventRecord(ev.e[3 + b], sc));
+    SQ_CUDA(cudaStreamWaitEvent(so, ev.e[3 + b], 0));
+    SQ_CUDA(cudaMemcpyAsync(ho + off, buf(b, 3), nb, cudaMemcpyDeviceToHost, so));
+    SQ_CUDA(cudaEventRecord(ev.e[5 + b], so));
+  }
+  // later work on `stream` (and a synchronisation of it) sees o complete: the copies out
+  // run in order on stream_out, so the last one's event covers them all
+  const int last = ((S + chunk - 1) / chunk - 1) & 1;
+  SQ_CUDA(cudaStreamWaitEvent(sc, ev.e[5 + last], 0));
+  return SQUAD_OK;
+}
+
 squad_status squad_attn_fwd_pass(const squad_desc* desc, int stage, const void* q, const void* k,
                                  const void* val, void* out, float* lse, void* stream) {
   Plan p;

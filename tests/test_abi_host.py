@@ -198,3 +198,34 @@ def test_multi_pass_workspace_size(lib):
     rows = 1 * 2 * 256
     # two bf16 upstream gradients, four fp32 accumulators, three fp32 row vectors
     assert got.value == 2 * rows * 128 * 2 + 4 * rows * 128 * 4 + 3 * rows * 4
+
+
+# ---------------------------------------------------------------- forward from host memory
+
+def test_host_forward_workspace_and_argument_errors(lib):
+    d = _desc(B=2, heads=3, T=4, H=8, W=8)          # 6 slices of 256 tokens, bf16, d = 128
+    got = ctypes.c_size_t(0)
+    assert lib.squad_attn_fwd_host_workspace_size(ctypes.byref(d), 4, ctypes.byref(got)) == OK
+    chunk = 4 * 256 * 128 * 2
+    fwd = ctypes.c_size_t(0)
+    dc = _desc(B=1, heads=4, T=4, H=8, W=8)
+    assert lib.squad_attn_workspace_size(ctypes.byref(dc), 0, ctypes.byref(fwd)) == OK
+    assert got.value == 2 * 4 * chunk + fwd.value     # two sets of q, k, v, o chunks + the chunk forward's
+    assert lib.squad_attn_fwd_host_workspace_size(ctypes.byref(d), 0, ctypes.byref(got)) == INVALID
+    assert lib.squad_attn_fwd_host_workspace_size(ctypes.byref(d), 4, None) == INVALID
+    big = ctypes.c_size_t(0)
+    assert lib.squad_attn_fwd_host_workspace_size(ctypes.byref(d), 100, ctypes.byref(big)) == OK  # capped at 6
+    need = ctypes.c_size_t(0)
+    assert lib.squad_attn_fwd_host_workspace_size(ctypes.byref(d), 4, ctypes.byref(need)) == OK
+    S1, S2, S3 = ctypes.c_void_p(0x20000), ctypes.c_void_p(0x30000), ctypes.c_void_p(0x40000)
+    def call(ws=FAKE, nb=None, s=(S1, S2, S3), q=FAKE, chunk=4):
+        return lib.squad_attn_fwd_host(ctypes.byref(d), q, FAKE, FAKE, FAKE, chunk, ws,
+                                       need.value if nb is None else nb, *s)
+    assert call(q=None) == INVALID
+    assert call(chunk=0) == INVALID
+    assert call(s=(S1, S2, S2)) == INVALID            # the three streams must differ
+    assert call(s=(S1, S1, S3)) == INVALID
+    assert call(s=(S1, None, S3)) == INVALID
+    assert call(ws=MISALIGNED) == ALIGN
+    assert call(ws=None) == WORKSPACE
+    assert call(nb=need.value - 16) == WORKSPACE

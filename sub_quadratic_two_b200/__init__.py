@@ -374,14 +374,16 @@ def _tiles_arg(tiles: Sequence[Sequence[int]]):
 
 
 def squad_attn_multi_fwd(q, k, v, grid, tiles, scale: Optional[float] = None,
-                         stream: Optional[torch.cuda.Stream] = None, one_launch: bool = True,
+                         stream: Optional[torch.cuda.Stream] = None, one_launch: Optional[bool] = None,
                          save: bool = True, out: Optional[torch.Tensor] = None,
                          workspace: Optional[torch.Tensor] = None):
     """k = len(tiles) + 1 passes over nested tiles (innermost first) through the C ABI.
 
     Returns (o, inter, lse): inter is [k-1, B, heads, n, d] (outputs of passes
     1..k-1), lse is [k, B, heads, n] fp32. one_launch: on bf16, run all passes in
-    one launch (passes a counter workspace); False runs one launch per pass.
+    one launch (passes a counter workspace); False runs one launch per pass; None
+    (default) picks one launch for save=False (same time, intermediates never
+    written to DRAM) and one launch per pass otherwise (measured 3% faster).
     save=False (inference): the intermediate outputs and the LSE are not kept
     (inter and lse are None; the intermediates live in the workspace and, on bf16,
     leave L2 without a write-back once read). out / workspace: optional
@@ -396,6 +398,8 @@ def squad_attn_multi_fwd(q, k, v, grid, tiles, scale: Optional[float] = None,
     o = torch.empty_like(q) if out is None else out
     inter = torch.empty((nt,) + tuple(q.shape), device=q.device, dtype=q.dtype) if save else None
     lse = torch.empty((nt + 1,) + tuple(q.shape[:3]), device=q.device, dtype=torch.float32) if save else None
+    if one_launch is None:
+        one_launch = not save
     ws, ws_n = None, 0
     if one_launch or not save:
         nb = ctypes.c_size_t(0)

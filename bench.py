@@ -175,7 +175,7 @@ def whole_job_throughput(world: int, flops_per_rank_step: float, ms_per_step: fl
     return world * flops_per_rank_step / (ms_per_step / 1e3) / 1e12
 
 
-FWD_KERNEL_SOURCES = ("squad_fwd_tc.cuh", "sm100.cuh", "geometry.h")
+FWD_KERNEL_SOURCES = ("squad_fwd_tc.cuh", "fwd_schedule.h", "sm100.cuh", "geometry.h")
 
 
 def code_only(text: str) -> str:

@@ -922,21 +922,7 @@ squad_status launch_fwd_multi(DeviceState* ds, int d, const MultiPlan& mp, const
   a.npass = np;
   a.bh = mp.gf[0].bh;
   a.lag = kMultiLag < a.bh ? kMultiLag : a.bh;
-  a.pref[0] = 0;
-  for (int j = 0; j < np; ++j) a.pref[j + 1] = a.pref[j] + a.ps[j].pairs_per_bh;
-  a.total_items = a.bh * a.pref[np];
-  // blocks 0 .. bh-1 + (np-1)*lag; block b holds pass j of head b - j*lag while that head
-  // exists, so blocks (np-1)*lag .. bh-1 hold every pass
-  const int first_full = (np - 1) * a.lag;
-  a.nmid = a.bh > first_full ? a.bh - first_full : 0;
-  a.lead_items = 0;
-  for (int b = 0; b < first_full; ++b)
-    for (int j = 0; j < np; ++j) {
-      const int h = b - j * a.lag;
-      if (h >= 0 && h < a.bh) a.lead_items += a.ps[j].pairs_per_bh;
-    }
-  a.f_full = sq::make_fastdiv(uint32_t(a.pref[np]));
-  a.f_n1 = a.f_n2 = a.f_n12 = a.f_full;  // unused in this mode
+  sq::plan_multi_order(a);
   a.scale_log2 = mp.base.scale * 1.4426950408889634f;
   a.counters = counters;
   a.err = ds->err;

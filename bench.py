@@ -424,9 +424,9 @@ def main():
         tiles3 = [(1, 1, 20), (1, 11, 20)]
         ws3 = torch.empty(sq.multi_fwd_workspace_size(q, wl.grid, tiles3, save=False), device=dev, dtype=torch.uint8)
         do3 = torch.randn_like(q)
-        for _ in range(2):  # launch order: inference form, training form, its backward (twice)
-            sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3, save=False, out=o, workspace=ws3)
-            mo, minter, mlse = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3)
+        for _ in range(2):  # launch order: inference form, training form (one launch each), backward (twice)
+            sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3, save=False, out=o, workspace=ws3, one_launch=True)
+            mo, minter, mlse = sq.squad_attn_multi_fwd(q, k, v, wl.grid, tiles3, one_launch=True)
             sq.squad_attn_multi_bwd(q, k, v, mo, minter, mlse, do3, wl.grid, tiles3)
             torch.cuda.synchronize()
         sq.poll_device_error()

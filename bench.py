@@ -60,7 +60,8 @@ def parse_args():
                     help="replicas: every rank runs the whole workload (independent problems, weak scaling); "
                          "sp: the workload's frames are sharded over the ranks and the two passes exchange rows "
                          "with NCCL all-to-alls (strong scaling)")
-    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--workload", default=None,
+                    help="workload name (default: the 27,280-token headline; long_video with --mode sp)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="skip the forward+backward training-step leg")
@@ -77,7 +78,10 @@ def parse_args():
     ap.add_argument("--profile", action="store_true",
                     help="profiling driver: one warm-up then one measured launch each of the fused forward, the "
                          "local pass alone and the global pass alone; no timing")
-    return ap.parse_args()
+    a = ap.parse_args()
+    if a.workload is None:
+        a.workload = "long_video" if a.mode == "sp" else HEADLINE
+    return a
 
 
 def load_peaks():

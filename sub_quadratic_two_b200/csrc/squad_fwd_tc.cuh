@@ -529,6 +529,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // Each thread holds its own row. A warp passes its 32 rows through a private
         // 128B-swizzled patch so that every global store writes four whole 128-byte lines.
         const float inv = 1.f / (l_run + lr_run);
+        const uint64_t inv2 = f2(inv, inv);
+        auto scale_pack = [&](uint32_t a0, uint32_t a1) -> uint32_t {
+          uint64_t m;
+          asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(m) : "l"(f2(__uint_as_float(a0), __uint_as_float(a1))), "l"(inv2));
+          return pack_bf16x2(f2_lo(m), f2_hi(m));
+        };
         const uint32_t xp = sbase + Lay::XP_OFF + (warp & 7) * 4096;
         const int lr = lane >> 3, lc = lane & 7;  // read-back: row 4*i + lr, 16-byte chunk lc
         int rtok[8];
@@ -544,11 +550,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           tmem_ld64(tO + h * 64, o);
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4),
-                         pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv));
+            st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4), scale_pack(o[8 * c + 0], o[8 * c + 1]),
+                         scale_pack(o[8 * c + 2], o[8 * c + 3]), scale_pack(o[8 * c + 4], o[8 * c + 5]),
+                         scale_pack(o[8 * c + 6], o[8 * c + 7]));
           __syncwarp();
 #pragma unroll
           for (int i = 0; i < 8; ++i) {

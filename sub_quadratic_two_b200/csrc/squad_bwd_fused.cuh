@@ -573,6 +573,7 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
     const uint32_t ds_row = sbase + Lay::DS_OFF + row * 128;
     const uint32_t xps = sbase + Lay::XPS_OFF + warp * 2048;
     const float c2 = args.scale_log2;
+    const uint64_t c2x2 = f2(c2, c2);
     const float log2e = 1.4426950408889634f;
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, to)) != 0;
@@ -614,8 +615,8 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         float* vl = vec + (t & 1u) * 256;
         const bool qlive = row < tile_valid_rows(g, qb) && (!PACKED || g.pk <= 1 || packed_row_live(g, j0, row));
         const int tok = qlive ? base + tile_row_offset(g, qb, row) : 0;
-        vl[row] = nx_lse;
-        vl[128 + row] = nx_d;
+        vl[row] = -nx_lse;  // negated: the gradient step adds them with paired instructions
+        vl[128 + row] = -nx_d;
         mbar_arrive(&bars[G_VEC]);
         if (!(ok = wwait(&bars[G_VEC], t & 1u))) break;
         if (!(ok = wwait(&bars[G_SFULL], t & 1u))) break;
@@ -630,23 +631,26 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
           uint32_t pk[16], dk[16];
 #pragma unroll
           for (int e4 = 0; e4 < 32; e4 += 4) {
+            // column statistics, negated: -lse * log2(e) and -D of the block's query columns
             const float4 lc4 = *reinterpret_cast<const float4*>(vl + c * 32 + e4);
             const float4 dc4 = *reinterpret_cast<const float4*>(vl + 128 + c * 32 + e4);
-            const float lcol[4] = {lc4.x, lc4.y, lc4.z, lc4.w};
-            const float dcol[4] = {dc4.x, dc4.y, dc4.z, dc4.w};
-            float p[4], dsv[4];
+            const uint64_t nl[2] = {f2(lc4.x, lc4.y), f2(lc4.z, lc4.w)};
+            const uint64_t nd[2] = {f2(dc4.x, dc4.y), f2(dc4.z, dc4.w)};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u2 = 0; u2 < 2; ++u2) {
+              const int e = e4 + 2 * u2;
+              const uint64_t x2 = ffma2(f2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2x2, nl[u2]);
               // key rows past the problem, and in a packed box the query columns of other
               // problems: P = dS = 0 (a select: exp2 of a zero score may overflow)
-              const bool same = !PACKED || ((pm >> (e4 + u)) & 1u);
-              p[u] = rlive && same ? ex2_approx(fmaf(__uint_as_float(s[e4 + u]), c2, -lcol[u])) : 0.f;
-              dsv[u] = p[u] * (__uint_as_float(dp[e4 + u]) - dcol[u]);
+              const bool same0 = !PACKED || ((pm >> e) & 1u), same1 = !PACKED || ((pm >> (e + 1)) & 1u);
+              const float p0 = rlive && same0 ? ex2_approx(f2_lo(x2)) : 0.f;
+              const float p1 = rlive && same1 ? ex2_approx(f2_hi(x2)) : 0.f;
+              const uint64_t d2 = fadd2(f2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), nd[u2]);
+              uint64_t ds2;
+              asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(ds2) : "l"(f2(p0, p1)), "l"(d2));
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+              dk[e >> 1] = pack_bf16x2(f2_lo(ds2), f2_hi(ds2));
             }
-            pk[e4 >> 1] = pack_bf16x2(p[0], p[1]);
-            pk[(e4 >> 1) + 1] = pack_bf16x2(p[2], p[3]);
-            dk[e4 >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-            dk[(e4 >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
           }
           tmem_st16(tS + c * 16, pk);
           // dS^T row: query columns [32c, 32c+32) are 16-byte chunks 4(c&1)..4(c&1)+3 of block c>>1

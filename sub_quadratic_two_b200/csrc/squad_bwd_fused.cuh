@@ -191,6 +191,27 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 
 enum { EPI_F32 = 0, EPI_BF16 = 1, EPI_RED = 2 };
 
+// Paired fp32 multiply (two lanes of one 64-bit register, rounded as two scalar multiplies).
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// The 16-byte chunk of scaled accumulator values v[0..3] for the transpose patch.
+__device__ __forceinline__ void st_scaled4(uint32_t addr, const uint32_t* v, uint64_t scale2) {
+  const uint64_t a = fmul2(f2(__uint_as_float(v[0]), __uint_as_float(v[1])), scale2);
+  const uint64_t b = fmul2(f2(__uint_as_float(v[2]), __uint_as_float(v[3])), scale2);
+  st_shared_v4(addr, uint32_t(a), uint32_t(a >> 32), uint32_t(b), uint32_t(b >> 32));
+}
+
+// x + a over a 16-byte chunk, in pairs.
+__device__ __forceinline__ float4 add4(const uint4& x, const float4& a) {
+  const uint64_t lo = fadd2(f2(__uint_as_float(x.x), __uint_as_float(x.y)), f2(a.x, a.y));
+  const uint64_t hi = fadd2(f2(__uint_as_float(x.z), __uint_as_float(x.w)), f2(a.z, a.w));
+  return make_float4(f2_lo(lo), f2_hi(lo), f2_lo(hi), f2_hi(hi));
+}
+
 // Drain one fp32 accumulator (D columns): value = acc * scale (+ add), then stored as
 // fp32 (EPI_F32) or bf16 (EPI_BF16), or added into fp32 memory (EPI_RED). The addend
 // loads of 64 columns are issued before their TMEM loads so the latencies overlap.
@@ -213,20 +234,17 @@ __device__ __forceinline__ void epi_acc(uint32_t taddr, uint32_t xp, int lane, c
     for (int rr = 0; rr < 2; ++rr) {
       uint32_t v[32];
       tmem_ld32(taddr + h * 64 + rr * 32, v);
+      const uint64_t scale2 = f2(scale, scale);
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        st_shared_v4(xp + lane * 128 + ((c ^ (lane & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * c]) * scale),
-                     __float_as_uint(__uint_as_float(v[4 * c + 1]) * scale),
-                     __float_as_uint(__uint_as_float(v[4 * c + 2]) * scale),
-                     __float_as_uint(__uint_as_float(v[4 * c + 3]) * scale));
+      for (int c = 0; c < 8; ++c) st_scaled4(xp + lane * 128 + ((c ^ (lane & 7)) << 4), v + 4 * c, scale2);
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 4 * i + lr;
         const uint4 x = ld_shared_v4(xp + r * 128 + ((lc ^ (r & 7)) << 4));
         if ((R.live >> r) & 1u) {
-          const float f0 = __uint_as_float(x.x) + a[rr][i].x, f1 = __uint_as_float(x.y) + a[rr][i].y;
-          const float f2 = __uint_as_float(x.z) + a[rr][i].z, f3 = __uint_as_float(x.w) + a[rr][i].w;
+          const float4 f = add4(x, a[rr][i]);
+          const float f0 = f.x, f1 = f.y, f2 = f.z, f3 = f.w;
           const size_t e = size_t(R.tok[i]) * D + h * 64 + rr * 32 + lc * 4;
           if (KIND == EPI_F32)
             *reinterpret_cast<float4*>(static_cast<float*>(out) + e) = make_float4(f0, f1, f2, f3);
@@ -273,12 +291,9 @@ __device__ __forceinline__ void epi_acc16(uint32_t taddr, uint32_t xp, int lane,
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
       if ((lane >> 4) == r) {
+        const uint64_t scale2 = f2(scale, scale);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(xp + prow * 128 + ((c ^ (prow & 7)) << 4), __float_as_uint(__uint_as_float(v[4 * c]) * scale),
-                       __float_as_uint(__uint_as_float(v[4 * c + 1]) * scale),
-                       __float_as_uint(__uint_as_float(v[4 * c + 2]) * scale),
-                       __float_as_uint(__uint_as_float(v[4 * c + 3]) * scale));
+        for (int c = 0; c < 8; ++c) st_scaled4(xp + prow * 128 + ((c ^ (prow & 7)) << 4), v + 4 * c, scale2);
       }
       __syncwarp();
 #pragma unroll
@@ -286,8 +301,8 @@ __device__ __forceinline__ void epi_acc16(uint32_t taddr, uint32_t xp, int lane,
         const int q = 4 * i + pr;
         const uint4 x = ld_shared_v4(xp + q * 128 + ((lc ^ (q & 7)) << 4));
         if ((live >> (16 * r + q)) & 1u) {
-          const float f0 = __uint_as_float(x.x) + a[r][i].x, f1 = __uint_as_float(x.y) + a[r][i].y;
-          const float f2 = __uint_as_float(x.z) + a[r][i].z, f3 = __uint_as_float(x.w) + a[r][i].w;
+          const float4 f = add4(x, a[r][i]);
+          const float f0 = f.x, f1 = f.y, f2 = f.z, f3 = f.w;
           const size_t e = size_t(tok[r][i]) * D + ch * 32 + lc * 4;
           if (KIND == EPI_F32)
             *reinterpret_cast<float4*>(static_cast<float*>(out) + e) = make_float4(f0, f1, f2, f3);

@@ -98,3 +98,13 @@ def test_forward_from_pageable_host_memory(cuda_ok):
                       slices_per_chunk=2)
     ref = sq.attention(*(t.cuda() for t in (inp.q, inp.k, inp.v)), wl.grid, wl.tile).cpu()
     assert torch.equal(out, ref)
+
+
+def test_forward_from_host_memory_batch_and_d64(cuda_ok):
+    # B = 2, 3 heads (6 slices in chunks of 4: one full, one ragged), d = 64
+    grid, tile = (4, 8, 8), (1, 4, 4)
+    inp = random_problem(83, 2, 3, 64, grid, tile, dtype=torch.bfloat16)
+    hq, hk, hv = (t.contiguous().pin_memory() for t in (inp.q, inp.k, inp.v))
+    out = sq.attention_host(hq, hk, hv, grid, tile, slices_per_chunk=4)
+    ref = sq.attention(*(t.cuda() for t in (inp.q, inp.k, inp.v)), grid, tile).cpu()
+    assert torch.equal(out, ref)

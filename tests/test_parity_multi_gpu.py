@@ -237,3 +237,20 @@ def test_three_passes_backward_full_size(cuda_ok):
         for name, a, b in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
             assert np.isfinite(_np(a[sel])).all(), name
             assert _err_scaled(_np(a[sel]), b) <= gmax, (h, name)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_packed_passes_batch_two_forward_and_backward(cuda_ok, d):
+    # B = 2 with packed boxes in both directions (20-token windows six to a box, 22-token
+    # groups five to a box): every (batch, head) slice against the oracle
+    grid, tiles = (4, 22, 40), [(1, 1, 20), (2, 11, 20)]
+    inp = random_problem(87, 2, 2, d, grid, (1, 1, 1), dtype=torch.bfloat16, with_do=True)
+    o, inter, lse, grads = _gpu_fwd_bwd(inp, grid, tiles)
+    ro, _, _, _ = oracle.squad_fwd_multi(inp.q, inp.k, inp.v, grid, tiles)
+    fmax, fmean, gmax = _bf16_tol(3)
+    mx, mean = _err(_np(o), ro)
+    assert mx <= fmax and mean <= fmean, (mx, mean)
+    ref = oracle.squad_bwd_multi(inp.q, inp.k, inp.v, inp.do, grid, tiles)
+    for name, a, b in zip(("dQ", "dK", "dV"), grads, ref):
+        assert np.isfinite(_np(a)).all(), name
+        assert _err(_np(a), b)[0] <= gmax, name

@@ -83,7 +83,11 @@ squad_status squad_attn_workspace_size(const squad_desc* desc, int which, size_t
  *   as one launch in which the global pass of each (batch, head) starts as
  *   soon as that head's local pass is done, while its Q, K and O1 are still in
  *   L2; the counters in the workspace order the two. When o1 is NULL, the
- *   local-pass rows are also dropped from L2 after their single use.
+ *   local-pass rows are also dropped from L2 after their single use. When the
+ *   Q, K and O1 rows of three (batch, head) slices (3 * 3 * n * d elements)
+ *   exceed 60% of the device's L2, the two passes run as two launches
+ *   instead, with the same results: the global pass would read them from DRAM
+ *   either way, and two launches then take less time.
  *   o1   : [B,heads,n,d] local-pass output, written when non-NULL (needed by
  *          the backward); when NULL the workspace holds it.
  *   lse1 : [B,heads,n] local-pass log-sum-exp, written when non-NULL.

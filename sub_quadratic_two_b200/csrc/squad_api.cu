@@ -51,6 +51,7 @@ squad_status cuda_fail(int code) {
 struct DeviceState {
   bool ready = false;
   int sms = 0;
+  int l2_bytes = 0;
   int* err = nullptr;          // device address of g_squad_dev_err
   bool fwd_attr_set[2][2] = {};  // [D=64/128][packed]
   bool fused_attr_set[2][2][2] = {};   // [D=64/128][out_f32][packed]
@@ -75,6 +76,7 @@ squad_status device_state(DeviceState** out) {
   DeviceState& s = g_dev[dev];
   if (!s.ready) {
     SQ_CUDA(cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev));
+    SQ_CUDA(cudaDeviceGetAttribute(&s.l2_bytes, cudaDevAttrL2CacheSize, dev));
     void* p = nullptr;
     SQ_CUDA(cudaGetSymbolAddress(&p, g_squad_dev_err));
     s.err = static_cast<int*>(p);
@@ -530,7 +532,13 @@ squad_status squad_attn_fwd(const squad_desc* desc, const void* q, const void* k
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int d = desc->d;
   if (desc->dtype == SQUAD_BF16) {
-    if (counters != nullptr) {
+    // One launch, the global pass of each head right behind its local pass, only pays when
+    // the heads in flight (the lag plus one) keep their Q, K and O1 in L2; otherwise (the
+    // 53,680-token shape: 3 x 41 MB) the global pass reads them from DRAM anyway and its
+    // waits on the local pass cost time, so the passes run as two launches.
+    const double head_bytes = 3.0 * double(p.g1.n) * d * p.elem;
+    const bool fits = (kFusedLag + 1) * head_bytes <= 0.6 * double(ds->l2_bytes);
+    if (counters != nullptr && fits) {
       // one launch: the global pass of each head runs right behind its local pass; without
       // a caller o1 the local-pass rows are dropped from L2 once the global pass has read them
       const bool drop = o1 == nullptr && (reinterpret_cast<uintptr_t>(o1buf) & 127u) == 0;

@@ -640,6 +640,16 @@ __global__ void __launch_bounds__(kBwdFusedThreads, 1)
         for (int c = 0; c < 4; ++c) {
           // this chunk's 32 query columns of the packed-box mask (selected, not indexed)
           const uint32_t pm = c == 0 ? pmask[0] : c == 1 ? pmask[1] : c == 2 ? pmask[2] : pmask[3];
+          if (PACKED && __all_sync(0xffffffffu, pm == 0u)) {
+            // no key row of this warp shares a problem with these query columns: P = dS = 0
+            tmem_st16_zero(tS + c * 16);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int chunk = (c & 1) * 4 + j;
+              st_shared_v4(ds_row + (c >> 1) * BLK + ((chunk ^ (row & 7)) << 4), 0u, 0u, 0u, 0u);
+            }
+            continue;
+          }
           uint32_t s[32], dp[32];
           tmem_ld32(tS + c * 32, s);
           tmem_ld32(tDP + c * 32, dp);

@@ -430,6 +430,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (32 * j + e >= lim) r[32 * j + e] = 0xff800000u;
           }
         }
+        // packed boxes: the 32-key chunks that hold a key of any row of this warp; the
+        // exponentials of the other chunks are skipped (their P is zero)
+        uint32_t wlive = 0xfu;
         if (PACKED && g.pk > 1) {
           // packed problems: keys of other problems in the box -> -inf. This row's problem
           // holds runs of pk_rowdiv columns, one run every pk * pk_rowdiv columns.
@@ -449,6 +452,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int e = 0; e < 128; ++e)
             if (!(((e < 64 ? mlo : mhi) >> (e & 63)) & 1ull)) r[e] = 0xff800000u;
+          const uint32_t mine = (uint32_t(mlo) != 0u ? 1u : 0u) | (uint32_t(mlo >> 32) != 0u ? 2u : 0u) |
+                                (uint32_t(mhi) != 0u ? 4u : 0u) | (uint32_t(mhi >> 32) != 0u ? 8u : 0u);
+          wlive = __reduce_or_sync(0xffffffffu, mine);
         }
         // row maximum: 8 independent partial maxima of three-input max
         float mp[8];
@@ -475,17 +481,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         uint64_t sl[2] = {0ull, 0ull};  // paired partial sums of p
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // two 64-column halves: P of a half is packed and stored at once
-          uint32_t pk[32];
+          if (!PACKED) {
+            uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const uint64_t x2 = ffma2(f2(__uint_as_float(r[64 * hh + e]), __uint_as_float(r[64 * hh + e + 1])),
-                                      c2x2, negx2);
-            const float p0 = ex2_approx(f2_lo(x2));
-            const float p1 = ex2_approx(f2_hi(x2));
-            sl[(e >> 1) & 1] = fadd2(sl[(e >> 1) & 1], f2(p0, p1));
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+            for (int e = 0; e < 64; e += 2) {
+              const uint64_t x2 = ffma2(f2(__uint_as_float(r[64 * hh + e]), __uint_as_float(r[64 * hh + e + 1])),
+                                        c2x2, negx2);
+              const float p0 = ex2_approx(f2_lo(x2));
+              const float p1 = ex2_approx(f2_hi(x2));
+              sl[(e >> 1) & 1] = fadd2(sl[(e >> 1) & 1], f2(p0, p1));
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+            tmem_st32(tS + hh * 32, pk);
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              if ((wlive >> (2 * hh + ch)) & 1u) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 32 * ch; e < 32 * ch + 32; e += 2) {
+                  const uint64_t x2 = ffma2(f2(__uint_as_float(r[64 * hh + e]), __uint_as_float(r[64 * hh + e + 1])),
+                                            c2x2, negx2);
+                  const float p0 = ex2_approx(f2_lo(x2));
+                  const float p1 = ex2_approx(f2_hi(x2));
+                  sl[(e >> 1) & 1] = fadd2(sl[(e >> 1) & 1], f2(p0, p1));
+                  pk[(e >> 1) - 16 * ch] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tS + hh * 32 + ch * 16, pk);
+              } else {
+                tmem_st16_zero(tS + hh * 32 + ch * 16);
+              }
+            }
           }
-          tmem_st32(tS + hh * 32, pk);
           if (hh == 0) {
             // O is rescaled before the first P.V half accumulates into it; the previous P.V
             // has completed (S of this step was issued after it)

@@ -610,8 +610,9 @@ def main():
         # groups of 20, 11 and 124 tokens. Inference form (intermediates in scratch, dropped
         # from L2 once read) and training form (intermediates and LSE kept for the backward),
         # each in one launch and in one launch per pass, interleaved call by call. Timed
-        # before the dense teacher below: after that library call the same launches ran
-        # 30% slower on the same box, even with its tensors freed.
+        # before the dense teacher below: in the first tens of milliseconds after that
+        # library call (seconds of full-power tensor work) the same launches ran 30-35%
+        # slower on the same box, and at normal speed again three seconds later.
         tiles3 = [(1, 1, 20), (1, 11, 20)]
         o3 = torch.empty_like(q)
         ws3 = torch.empty(sq.multi_fwd_workspace_size(q, wl.grid, tiles3, save=False), device=dev, dtype=torch.uint8)

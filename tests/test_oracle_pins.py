@@ -266,6 +266,35 @@ def test_backward_matches_autograd_of_masked_dense(grid, tile):
     np.testing.assert_allclose(dv, v.grad.numpy(), rtol=0, atol=1e-11)
 
 
+def _random_geometries(count, seed):
+    """Seeded grids (each side 1..9) with a random divisor of each side as the window tile."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < count:
+        grid = tuple(int(x) for x in rng.integers(1, 10, size=3))
+        if math.prod(grid) > 360:
+            continue
+        tile = tuple(int(rng.choice([t for t in range(1, g + 1) if g % t == 0])) for g in grid)
+        out.append((grid, tile, int(rng.integers(1, 9))))
+    return out
+
+
+@pytest.mark.parametrize("grid,tile,d", _random_geometries(24, 20261203))
+def test_forward_and_backward_equal_masked_dense_on_random_geometries(grid, tile, d):
+    # a sweep over seeded random grids and tiles (windows of one token, whole-grid windows,
+    # tT > 1, odd sides): forward against the masked library SDPA, backward against autograd
+    inp = random_problem(73, 1, 2, d, grid, tile, dtype=torch.float64, with_do=True)
+    q, k, v = (x.clone().requires_grad_(True) for x in (inp.q, inp.k, inp.v))
+    ref_o, ref_o1 = _masked_sdpa_two_pass(q, k, v, grid, tile)
+    (ref_o * inp.do).sum().backward()
+    o, o1, _, _, _ = oracle.squad_fwd(inp.q, inp.k, inp.v, grid, tile)
+    np.testing.assert_allclose(o1, ref_o1.detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o, ref_o.detach().numpy(), rtol=0, atol=1e-12)
+    dq, dk, dv = oracle.squad_bwd(inp.q, inp.k, inp.v, inp.do, grid, tile)
+    for name, got, t in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        np.testing.assert_allclose(got, t.grad.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
 def test_bad_shapes_rejected():
     inp = random_problem(81, 1, 1, 4, (2, 4, 4), (1, 2, 2), dtype=torch.float64)
     with pytest.raises(ValueError):

@@ -105,6 +105,41 @@ def test_passes_equal_masked_dense_attention(grid, tiles):
     np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
 
 
+def _random_chains(count, seed):
+    """Seeded grids (sides 1..8) with chains of 1-3 nested tiles (each a divisor chain)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < count:
+        grid = tuple(int(x) for x in rng.integers(1, 9, size=3))
+        if int(np.prod(grid)) > 256:
+            continue
+        ntiles = int(rng.integers(1, 4))
+        tiles, cur = [], (1, 1, 1)
+        for _ in range(ntiles):
+            # the next tile: a multiple of the current one that divides the grid
+            nxt = tuple(int(rng.choice([t for t in range(c, g + 1) if t % c == 0 and g % t == 0]))
+                        for c, g in zip(cur, grid))
+            tiles.append(nxt)
+            cur = nxt
+        out.append((grid, tiles, int(rng.integers(1, 7))))
+    return out
+
+
+@pytest.mark.parametrize("grid,tiles,d", _random_chains(16, 1203))
+def test_random_chains_equal_masked_dense_forward_and_backward(grid, tiles, d):
+    # seeded random grids and tile chains (repeated tiles, one-token tiles, whole-grid
+    # tiles): forward against masked SDPA composed pass by pass, backward against autograd
+    q, k, v, do = _problem(8, grid, d=d)
+    qq, kk, vv = (t.clone().requires_grad_(True) for t in (q, k, v))
+    ref = _masked_dense_passes(qq, kk, vv, grid, tiles)
+    (ref * do).sum().backward()
+    o, _, _, _ = oracle.squad_fwd_multi(q, k, v, grid, tiles)
+    np.testing.assert_allclose(o, ref.detach().numpy(), rtol=0, atol=1e-12)
+    g = oracle.squad_bwd_multi(q, k, v, do, grid, tiles)
+    for name, a, b in zip(("dq", "dk", "dv"), g, (qq.grad, kk.grad, vv.grad)):
+        np.testing.assert_allclose(a, b.numpy(), rtol=0, atol=1e-11, err_msg=name)
+
+
 def test_mac_count_closed_form():
     # 2 n d sum_j |t_j| / |t_{j-1}| per (batch, head): scores plus value sums
     grid, tiles = (2, 4, 8), [(1, 2, 2), (2, 2, 4)]

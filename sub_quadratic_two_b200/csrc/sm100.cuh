@@ -241,7 +241,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-// 32 registers per thread -> 32 lanes x 32 columns of TMEM (no wait).
 // 16 zero columns (every operand the zero register)
 __device__ __forceinline__ void tmem_st16_zero(uint32_t taddr) {
   const uint32_t z = 0u;
@@ -252,6 +251,7 @@ __device__ __forceinline__ void tmem_st16_zero(uint32_t taddr) {
       : "memory");
 }
 
+// 32 registers per thread -> 32 lanes x 32 columns of TMEM (no wait).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
